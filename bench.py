@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Benchmark of the MoBA hot path on B200.
+
+One step = the whole hot path over one batch of synthetic input: key conv +
+centroids, routing + top-k, block index, sparse attention forward and
+normalisation, then the backward (preprocess, block index, attention, dQ).
+Default workload: N = 64K tokens, 16 heads, d = 64, B = 32, top-k = 32, key
+conv width 4, 256 planted needles per head (the small-block long-context
+shape).  The JSON line reports effective TFLOP/s on the nominal FLOP count
+3.5 * 4*N*H*k*B*d (forward 4*N*H*k*B*d, backward 2.5x that) and its
+fraction of the measured B200 bf16 tensor peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun) every rank runs its own independent
+problem of the same shape (different seeds): no data-path collective; the
+step time is the max over ranks and ``value`` the aggregate throughput.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from block_sparse_long_key_b200 import synth  # noqa: E402
+
+METRIC = "MoBA fwd/bwd effective TFLOP/s & ms at N=64K,B=32; % of B200 bf16 tensor peak"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch of each kernel, read from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
+# kernel source file it was taken with: a changed source voids the figure.
+NCU_TRAFFIC = {}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def src_sha(fname):
+    with open(os.path.join(ROOT, "block_sparse_long_key_b200", "csrc", fname), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        maxclk = max(r[1] for r in rows)
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": maxclk, "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max(value: float, device, world: int) -> float:
+    """Max of a float over ranks (identity for one rank)."""
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(flops_per_step_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank's work over the slowest rank's time."""
+    return flops_per_step_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
+def rank_seed(w: synth.Workload, rank: int) -> int:
+    return w.seed + 7919 * rank
+
+
+def stage_roofline(name, w, pairs, scored, peaks):
+    """(bound, algorithmic amount per launch, unit) of one stage."""
+    T, hq, hkv, d, B = w.total_tokens, w.h_q, w.h_kv, w.head_dim, w.block_size
+    if name == "fwd_attn":
+        return "tensor", 4.0 * B * d * pairs, "flop"
+    if name == "bwd_attn":
+        return "tensor", 10.0 * B * d * pairs, "flop"
+    if name == "fwd_route":
+        return "tensor", 2.0 * 2.0 * d * scored, "flop"   # hi + lo products
+    if name == "fwd_centroid":
+        return "hbm", T * hkv * d * 2.0 * (3 if w.conv_width else 1), "byte"
+    if name == "fwd_finalize":
+        return "hbm", T * hq * (d * 6.0 + 12), "byte"
+    if name == "bwd_pre":
+        return "hbm", T * hq * (d * 8.0 + 4), "byte"
+    if name == "bwd_dq":
+        return "hbm", T * hq * d * 6.0, "byte"
+    if name in ("fwd_index", "bwd_index"):
+        return "hbm", T * hq * w.topk * 4.0 * 2 + pairs * 4.0 * 3, "byte"
+    return "hbm", 0.0, "byte"
+
+
+KERNEL_SRC = {"fwd_attn": "fwd.cu", "bwd_attn": "bwd.cu", "fwd_route": "route.cu", "fwd_centroid": "conv_centroid.cu",
+              "fwd_finalize": "fwd.cu", "bwd_pre": "bwd.cu", "bwd_dq": "bwd.cu", "fwd_index": "index.cu",
+              "bwd_index": "index.cu"}
+
+# Kernels of ours launched per step: forward 9 (plan, conv/centroid, route,
+# count, scan, fill, attention, finalize, fallback), backward 7 (plan, count,
+# scan, fill, preprocess, attention, dQ).
+LAUNCHES_PER_STEP = 16
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) timing
+
+def oracle_sample(w: synth.Workload, seed: int, rows_per_step: int, steps: int, warmup: int):
+    """Times the fp64 oracle on sampled query rows.  Returns per-step TFLOP/s
+    values and a description.  Routing, attention and the per-row backward
+    run inside the timed region; the key conv and centroids (O(N d), computed
+    once for the whole input) are prepared outside it."""
+    from oracle import moba_oracle as orc
+
+    x = synth.make_inputs(w, seed=seed)
+    cu = x["cu_seqlens"].numpy()
+    q = x["q"].double().numpy()
+    k = x["k"].double().numpy()
+    if "conv_w" in x:
+        k = orc.key_conv(k, x["conv_w"].double().numpy(), cu)
+    v = x["v"].double().numpy()
+    dout = x["dout"].double().numpy()
+    cents = orc.block_centroids(k, cu, w.block_size)
+    r = np.random.default_rng(seed)
+    vals = []
+    cpu0, wall0 = time.process_time(), time.perf_counter()
+    for step in range(warmup + steps):
+        ts = r.integers(0, w.total_tokens, rows_per_step)
+        hs = r.integers(0, w.h_q, rows_per_step)
+        rows = list(zip(ts.tolist(), hs.tolist()))
+        t0 = time.perf_counter()
+        sel = np.full((w.total_tokens, w.h_q, w.topk), -1, dtype=np.int64)
+        starts = cu[:-1]
+        g = w.h_q // w.h_kv
+        useful = 0.0
+        for t, h in rows:
+            s = int(np.searchsorted(starts, t, side="right") - 1)
+            blocks, _ = orc.route_row(q[t, h], cents[s][h // g], t - int(cu[s]), w.block_size, w.topk)
+            sel[t, h, :len(blocks)] = blocks
+            useful += 3.5 * 4.0 * w.topk * w.block_size * w.head_dim
+        orc.attention(q, k, v, sel, cu, w.block_size, rows=rows)
+        orc.backward_rows(q, k, v, dout, sel, cu, w.block_size, rows)
+        dt = time.perf_counter() - t0
+        if step >= warmup:
+            vals.append(useful / dt / 1e12)
+    cores = max(1, round((time.process_time() - cpu0) / max(time.perf_counter() - wall0, 1e-9)))
+    desc = ("%d random (query, head) rows per step: routing against all past centroids, attention and the "
+            "per-row backward in fp64 numpy; FLOPs counted as 3.5*4*k*B*d per row (nominal, as on the GPU); "
+            "key conv and centroids prepared outside the timed region" % rows_per_step)
+    return vals, desc, cores
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    from block_sparse_long_key_b200 import moba
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[args.workload]
+    peaks, peak_src = load_peaks()
+    moba.lib()
+
+    seed = rank_seed(w, rank)
+    x = synth.make_inputs(w, seed=seed)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    T, hq, hkv, d, B, topk = w.total_tokens, w.h_q, w.h_kv, w.head_dim, w.block_size, w.topk
+    shape = moba.shape_of(g["q"], g["k"], g["cu_seqlens"], B, topk)
+    ws_f = moba.alloc_workspace(moba.fwd_workspace_size(shape), dev)
+    ws_b = moba.alloc_workspace(moba.bwd_workspace_size(shape), dev)
+    out = torch.empty_like(g["q"])
+    lse = torch.empty((T, hq), dtype=torch.float32, device=dev)
+    sel = torch.empty((T, hq, topk), dtype=torch.int32, device=dev)
+    kc = torch.empty_like(g["k"]) if w.conv_width else None
+    dq, dk, dv = torch.empty_like(g["q"]), torch.empty_like(g["k"]), torch.empty_like(g["v"])
+    conv_w = g.get("conv_w")
+
+    def step(qd, kd, vd, dod, cud, cw):
+        _, _, _, k_used = moba.forward(qd, kd, vd, cud, B, topk, conv_w=cw, workspace=ws_f, out=out, lse=lse,
+                                       sel_idx=sel, k_conv=kc)
+        moba.backward(qd, k_used, vd, out, lse, dod, sel, cud, B, workspace=ws_b, dq=dq, dk=dk, dv=dv)
+
+    for _ in range(args.warmup):
+        step(g["q"], g["k"], g["v"], g["dout"], g["cu_seqlens"], conv_w)
+    torch.cuda.synchronize()
+    status = moba.check_status(ws_f) | moba.check_status(ws_b)
+    pairs = int((sel >= 0).sum().item())
+    pos = torch.cat([torch.arange(b - a) for a, b in zip(x["cu_seqlens"][:-1].tolist(),
+                                                         x["cu_seqlens"][1:].tolist())]).double()
+    scored = float((pos // B).sum().item()) * hq
+
+    stream = torch.cuda.current_stream()
+    stage_sets = [moba.StageEvents() for _ in range(args.steps)]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        ev0.record(stream)
+        for i in range(args.steps):
+            with stage_sets[i]:
+                step(g["q"], g["k"], g["v"], g["dout"], g["cu_seqlens"], conv_w)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_max = reduce_max(ms, dev, world)
+    stage_ms = {}
+    for s in moba.STAGES:
+        stage_ms[s] = statistics.mean(e.ms()[s] for e in stage_sets)
+    fwd_ms = sum(v for k_, v in stage_ms.items() if k_.startswith("fwd"))
+    bwd_ms = sum(v for k_, v in stage_ms.items() if k_.startswith("bwd"))
+
+    flops = w.fwd_flops() + w.bwd_flops()
+    value = aggregate_value(flops, world, ms_max)
+    peak_t = float(peaks["bf16_tflops"])
+
+    dom = max(stage_ms, key=stage_ms.get)
+    bound, amount, unit = stage_roofline(dom, w, pairs, scored, peaks)
+    if bound == "tensor":
+        achieved = amount / (stage_ms[dom] * 1e-3) / 1e12
+        peak, runit = peak_t, "TFLOP/s"
+    else:
+        achieved = amount / (stage_ms[dom] * 1e-3) / 1e9
+        peak, runit = float(peaks["hbm_gbs"]), "GB/s"
+    tr = NCU_TRAFFIC.get(dom)
+    traffic = tr["bytes"] if tr and tr.get("sha") == src_sha(KERNEL_SRC.get(dom, "fwd.cu")) else None
+    roofline = {"kernel": dom, "bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": runit,
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": "%s (MEASURED_PEAKS.json burst)" % peak_src if bound == "tensor" else peak_src,
+                "per_unit": ("%s per (query, head, block) pair; %d pairs per launch" %
+                             ("4*B*d FLOP" if dom == "fwd_attn" else "10*B*d FLOP", pairs))
+                if dom in ("fwd_attn", "bwd_attn") else unit}
+
+    # End to end through the public API with host buffers.
+    e2e = None
+    if not args.no_e2e:
+        names_in = ["q", "k", "v", "dout"] + (["conv_w"] if conv_w is not None else []) + ["cu_seqlens"]
+        host = {n: x[n].pin_memory() for n in names_in}
+        dev_in = {n: torch.empty_like(g[n]) for n in names_in}
+        outs = [out, lse, dq, dk, dv]
+        host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = sum(t.numel() * t.element_size() for t in outs)
+        ne = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            for n in names_in:
+                dev_in[n].copy_(host[n], non_blocking=True)
+            step(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["dout"], dev_in["cu_seqlens"], dev_in.get("conv_w"))
+            for t, h in zip(outs, host_out):
+                h.copy_(t, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(ne):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = reduce_max(e0.elapsed_time(e1) / ne, dev, world)
+        e2e = {"value": round(aggregate_value(flops, world, ems), 3), "unit": UNIT, "ms_per_step": round(ems, 3),
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": ne}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        vals, desc, cores = oracle_sample(w, seed, args.cpu_rows, 2, 1)
+        cpu = {"value": round(statistics.mean(vals), 9), "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": desc}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        in_bytes = sum(g[n].numel() * g[n].element_size() for n in ("q", "k", "v", "dout"))
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "seq_len": T, "batch": w.batch, "h_q": hq, "h_kv": hkv, "head_dim": d,
+                       "block_size": B, "topk": topk, "conv_width": w.conv_width,
+                       "needles_per_head": w.needles_per_head,
+                       "l2": "inputs %.0f MB > %d MB L2 (no flush)" % (in_bytes / 1e6, L2_BYTES >> 20),
+                       "parallelism": "independent problem per GPU" if world > 1 else "single GPU"},
+            "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
+            "fwd_tflops": round(w.fwd_flops() / (fwd_ms * 1e-3) / 1e12, 3),
+            "bwd_tflops": round(w.bwd_flops() / (bwd_ms * 1e-3) / 1e12, 3),
+            "pct_of_bf16_peak": round(100.0 * value / world / peak_t, 3),
+            "peak_bf16_tflops": peak_t, "peak_source": peak_src,
+            "stage_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
+            "pairs": pairs, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks.summary(), "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    vals, desc, cores = oracle_sample(w, w.seed, args.ref_rows, args.steps, args.warmup)
+    v = statistics.mean(vals)
+    flops_row = 3.5 * 4.0 * w.topk * w.block_size * w.head_dim
+    ms = args.ref_rows * flops_row / (v * 1e12) * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 9), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "seq_len": w.total_tokens, "batch": w.batch, "h_q": w.h_q,
+                       "h_kv": w.h_kv, "head_dim": w.head_dim, "block_size": w.block_size, "topk": w.topk,
+                       "conv_width": w.conv_width, "needles_per_head": w.needles_per_head,
+                       "sample_rows_per_step": args.ref_rows},
+            "cpu_baseline": {"value": round(v, 9), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(v, 9), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(synth.WORKLOADS), default=synth.HEADLINE)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=1500, help="oracle rows per CPU-baseline step")
+    ap.add_argument("--ref-rows", type=int, default=400, help="oracle rows per --impl reference step")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,68 @@
+// Internal launchers of the MoBA kernels.  Every launcher enqueues work on
+// `st` and returns the launch status; none of them allocates or
+// synchronises.  Pointers are device pointers; layouts are documented in
+// include/moba.h and at each kernel.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moba {
+
+typedef __nv_bfloat16 bf16;
+
+// Query rows per routing tile.
+constexpr int kRouteTile = 64;
+
+struct SeqPlan {
+  const int32_t* cu;        // sanitised cu_seqlens [batch + 1]
+  const int32_t* blk_off;   // first global block of each sequence [batch + 1]
+  const int32_t* tile_off;  // first routing tile of each sequence [batch + 1]
+  int batch;
+  int total_tokens;
+  int nb_max;               // static bound on the number of blocks
+};
+
+cudaError_t launch_plan(const int32_t* cu_in, int batch, int total_tokens, int block_size,
+                        int32_t* cu_out, int32_t* blk_off, int32_t* tile_off, int32_t* status,
+                        cudaStream_t st);
+
+cudaError_t launch_conv_centroid(const bf16* k, const float* conv_w, int conv_width, const SeqPlan& p,
+                                 int h_kv, int d, int block_size, bf16* k_out, float* cent,
+                                 bf16* cent_hi, bf16* cent_lo, cudaStream_t st);
+
+cudaError_t launch_route(const bf16* q, const bf16* k, const bf16* cent_hi, const bf16* cent_lo,
+                         const SeqPlan& p, int h_q, int h_kv, int d, int block_size, int topk,
+                         int32_t* sel_idx, float* mref, int32_t* flag, float* lacc, float* oacc,
+                         cudaStream_t st);
+
+cudaError_t launch_build_index(const int32_t* sel_idx, const SeqPlan& p, int h_q, int h_kv,
+                               int block_size, int topk, int32_t* cnt, int32_t* ptr, int32_t* cursor,
+                               int32_t* rows, int32_t* status, cudaStream_t st);
+
+cudaError_t launch_fwd_attn(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p,
+                            const int32_t* ptr, const int32_t* rows, const float* mref, int h_q,
+                            int h_kv, int d, int block_size, float* oacc, float* lacc, int32_t* flag,
+                            cudaStream_t st);
+
+cudaError_t launch_fwd_finalize(const float* oacc, const float* lacc, const float* mref,
+                                const int32_t* flag, int nrows, int d, bf16* out, float* lse,
+                                int32_t* flag_list, cudaStream_t st);
+
+cudaError_t launch_fwd_fallback(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p,
+                                const int32_t* sel_idx, const int32_t* flag_list, int h_q, int h_kv,
+                                int d, int block_size, int topk, bf16* out, float* lse,
+                                cudaStream_t st);
+
+cudaError_t launch_bwd_pre(const bf16* out, const bf16* dout, int nrows, int d, float* dsum,
+                           float* dqacc, cudaStream_t st);
+
+cudaError_t launch_bwd_attn(const bf16* q, const bf16* k, const bf16* v, const bf16* dout,
+                            const float* lse, const float* dsum, const SeqPlan& p, const int32_t* ptr,
+                            const int32_t* rows, int h_q, int h_kv, int d, int block_size,
+                            float* dqacc, bf16* dk, bf16* dv, cudaStream_t st);
+
+cudaError_t launch_bwd_dq(const float* dqacc, int n, bf16* dq, cudaStream_t st);
+
+}  // namespace moba

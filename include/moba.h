@@ -1,0 +1,209 @@
+/*
+ * moba.h - C ABI of the B200 (sm_100a) MoBA hot path.
+ *
+ * MoBA (Mixture of Block Attention), as defined in "Optimizing Mixture of
+ * Block Attention" (Xiao, Guo, Mazaheri, Han; summarised on the lowest.today
+ * pages, Italian and German): keys are split into blocks of B tokens, each
+ * block is represented by its mean key (centroid), every query scores the
+ * causally visible centroids with q . k~_j, keeps its own block plus the
+ * best-scoring earlier blocks (k blocks in all), and exact softmax attention
+ * with scale 1/sqrt(d) runs over the selected tokens only.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  Tokens are packed ("varlen"): sequences s = 0..batch-1 occupy tokens
+ *  [cu_seqlens[s], cu_seqlens[s+1]).  cu_seqlens is int32 [batch + 1] in
+ *  DEVICE memory, non-decreasing, cu_seqlens[0] = 0, cu_seqlens[batch] = T.
+ *  Blocks, causality and the key convolution restart at every sequence.
+ *
+ *  q, out, dout, dq:  bf16 [T, h_q,  d] row-major (d contiguous).
+ *  k, v, dk, dv:      bf16 [T, h_kv, d] row-major.
+ *  lse:               fp32 [T, h_q], natural log of sum exp(q.k/sqrt(d)).
+ *  sel_idx:           int32 [T, h_q, topk]: the selected blocks of each
+ *                     query, block numbers relative to the query's sequence,
+ *                     sorted ascending, the query's own block last among the
+ *                     valid entries, unused slots -1.
+ *  Query head h reads KV head h / (h_q / h_kv) (grouped-query attention).
+ *
+ *  Every pointer is a device pointer owned by the caller, 16-byte aligned
+ *  (the workspace: 256-byte aligned).  The library allocates no memory, keeps
+ *  no state between calls (apart from the optional per-thread stage-timing
+ *  table of moba_set_stage_events) and never synchronises: each call only enqueues
+ *  kernels on `stream` (a cudaStream_t; NULL = legacy default stream) and
+ *  returns.  Argument errors are reported synchronously by the return code;
+ *  data-dependent errors found on the device (bad cu_seqlens, out-of-range
+ *  sel_idx entries) are recorded in the workspace's status word and read
+ *  with moba_check_status().  No call ever traps the device.
+ *
+ *  Supported sizes: d in {64, 128}; B in {16, 32, 64, 128}; 1 <= topk <= 64;
+ *  h_q a multiple of h_kv; T * h_q * max(d, topk) < 2^31.  T = 0 is valid:
+ *  the call returns MOBA_OK after checking the shape, launches nothing and
+ *  leaves the workspace (and its status word) untouched.
+ */
+#ifndef MOBA_H_
+#define MOBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Problem shape.  All fields are plain host values. */
+typedef struct moba_shape {
+  int32_t total_tokens; /* T = cu_seqlens[batch] */
+  int32_t batch;        /* number of packed sequences, >= 1 */
+  int32_t h_q;          /* query heads */
+  int32_t h_kv;         /* key/value heads; divides h_q */
+  int32_t head_dim;     /* d: 64 or 128 */
+  int32_t block_size;   /* B: 16, 32, 64 or 128 */
+  int32_t topk;         /* k: selected blocks per query, own block included */
+} moba_shape;
+
+/* Return codes. */
+#define MOBA_OK 0
+#define MOBA_EINVAL (-1)     /* null pointer, unsupported size, bad shape */
+#define MOBA_EALIGN (-2)     /* pointer not 16-byte (workspace: 256-byte) aligned */
+#define MOBA_EWORKSPACE (-3) /* workspace smaller than the *_workspace_size() */
+#define MOBA_ELAUNCH (-4)    /* a kernel launch failed (CUDA error) */
+#define MOBA_EDEVICE (-5)    /* moba_check_status(): the device flagged bad input */
+
+/* Device status bits reported by moba_check_status(). */
+#define MOBA_STATUS_BAD_SEQLENS 1 /* cu_seqlens not monotone or not ending at T */
+#define MOBA_STATUS_BAD_SEL_IDX 2 /* a sel_idx entry outside [-1, own block]; skipped */
+#define MOBA_STATUS_INDEX_OVERFLOW 4
+
+/* Bytes of device workspace moba_forward / moba_key_conv_centroid need for
+ * `shape` (0 for an invalid shape).  The caller allocates it; its contents
+ * need no initialisation and are scratch after the call, except the status
+ * word read by moba_check_status(). */
+size_t moba_fwd_workspace_size(const moba_shape* shape);
+
+/* Bytes of device workspace moba_backward / moba_build_index need. */
+size_t moba_bwd_workspace_size(const moba_shape* shape);
+
+/*
+ * Key convolution (optional) and block centroids: the first two steps of
+ * the forward, exposed on their own.
+ *
+ * Follows "Optimizing Mixture of Block Attention", section "Progettazione
+ * della Convoluzione delle Chiavi (Appendice B)", "Forma Formale":
+ *   k'_t = k_t + SiLU(sum_{l=0}^{W-1} w_l (.) k_{t-l})
+ * depthwise (one filter per channel), causal with zero padding before the
+ * sequence start, no bias; k' is rounded to bf16 (nearest even).  And section
+ * "Architettura del Modello Statistico" 1: centroid of block j = mean of its
+ * keys (k' when the conv is on; a partial last block averages its real
+ * tokens).
+ *
+ *  k         bf16 [T, h_kv, d]   input keys
+ *  conv_w    fp32 [h_kv, d, conv_width], tap l multiplies k_{t-l}; NULL and
+ *            conv_width = 0 for no convolution; conv_width <= 8
+ *  k_out     bf16 [T, h_kv, d]   k' (ignored when conv_width = 0); must not
+ *            alias k
+ *  centroid  fp32 [h_kv, nblk, d] where block j of sequence s is row
+ *            blk_off[s] + j, blk_off[s] = sum_{s'<s} ceil(L_s'/B), and
+ *            nblk = T / B + batch is the row capacity (unused rows untouched)
+ */
+int moba_key_conv_centroid(const void* k, const float* conv_w, int conv_width, const int32_t* cu_seqlens,
+                           const moba_shape* shape, void* k_out, float* centroid, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
+ * MoBA forward: (key conv) -> centroids -> routing + top-k -> block index ->
+ * gather-and-densify sparse attention -> normalisation.
+ *
+ * Routing: "Optimizing Mixture of Block Attention", section "Architettura del
+ * Modello Statistico" 1 (s_j = q . k~_j) and "Definizione del Compito"
+ * (top-k blocks); a query at local position p (block b = p / B) scores blocks
+ * j < b, keeps the topk-1 best (exact ties: lower j) and always its own block.
+ * Attention: "Definizione del Compito", O = softmax(Q K^T / sqrt(d)) V over
+ * the selected tokens, causal inside the own block.
+ *
+ *  q, k, v           inputs (see conventions)
+ *  conv_w, conv_width optional key convolution, as in moba_key_conv_centroid;
+ *                    when on, k_conv_out (bf16 [T, h_kv, d]) receives k',
+ *                    which routing and attention use and which the backward
+ *                    must be given as its k
+ *  out               bf16 [T, h_q, d]
+ *  lse               fp32 [T, h_q]
+ *  sel_idx           int32 [T, h_q, topk] (output)
+ *  workspace         >= moba_fwd_workspace_size(shape) bytes
+ */
+int moba_forward(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                 const moba_shape* shape, const float* conv_w, int conv_width, void* k_conv_out, void* out,
+                 float* lse, int32_t* sel_idx, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Block index: inverts sel_idx (query -> blocks) into per-(KV head, block)
+ * query lists, the key-block-major varlen layout of "Optimizing Mixture of
+ * Block Attention", section "Progettazione del Kernel FlashMoBA", "Tre Kernel
+ * Fusi" 1 (stage 3) used by the forward and the backward.
+ *
+ *  blk_ptr   int32 [h_kv * nblk + 1]: bucket (kvh, gb) = kvh * nblk + gb
+ *            holds entries blk_ptr[b] .. blk_ptr[b+1]-1; nblk = T / B + batch
+ *  blk_rows  int32 [T * h_q * topk] capacity: query row ids t * h_q + h of
+ *            every valid pick (own block included); order inside a bucket
+ *            is unspecified
+ */
+int moba_build_index(const int32_t* sel_idx, const int32_t* cu_seqlens, const moba_shape* shape,
+                     int32_t* blk_ptr, int32_t* blk_rows, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
+/*
+ * MoBA backward with the selection held fixed ("Optimizing Mixture of Block
+ * Attention", section "Progettazione del Kernel FlashMoBA", "Tre Kernel
+ * Fusi" 3: recompute per key block, dQ by atomic accumulation in fp32).
+ *
+ *  q, k, v, out, lse, sel_idx   as given to / returned by moba_forward (k is
+ *                               k' when the forward used the key conv)
+ *  dout              bf16 [T, h_q, d]
+ *  dq                bf16 [T, h_q, d]  (output)
+ *  dk, dv            bf16 [T, h_kv, d] (output; summed over the query heads
+ *                    of each group).  The gradient stops at k': the key
+ *                    convolution's own backward is not part of this call.
+ *  workspace         >= moba_bwd_workspace_size(shape) bytes
+ */
+int moba_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                  const void* dout, const int32_t* sel_idx, const int32_t* cu_seqlens, const moba_shape* shape,
+                  void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Optional stage timing for benchmarks.  While a table is installed on the
+ * calling host thread, moba_forward and moba_backward record events[2*i]
+ * (a cudaEvent_t) on their stream before stage i and events[2*i+1] after it,
+ * for every i with 2*i+1 < n_events; NULL entries are skipped.  The stages:
+ * forward plan, key conv + centroids, routing, block index, attention,
+ * normalisation (+ exact re-computation of flagged rows); backward plan,
+ * block index, preprocessing, attention, dQ conversion.  The table is read,
+ * never written; the caller keeps it (and the events) alive while installed.
+ * Pass (NULL, 0) to remove it.  Results are unaffected.
+ */
+#define MOBA_STAGE_FWD_PLAN 0
+#define MOBA_STAGE_FWD_CENTROID 1
+#define MOBA_STAGE_FWD_ROUTE 2
+#define MOBA_STAGE_FWD_INDEX 3
+#define MOBA_STAGE_FWD_ATTN 4
+#define MOBA_STAGE_FWD_FINALIZE 5
+#define MOBA_STAGE_BWD_PLAN 6
+#define MOBA_STAGE_BWD_INDEX 7
+#define MOBA_STAGE_BWD_PRE 8
+#define MOBA_STAGE_BWD_ATTN 9
+#define MOBA_STAGE_BWD_DQ 10
+#define MOBA_NUM_STAGES 11
+int moba_set_stage_events(void* const* events, int n_events);
+
+/* Synchronises `stream`, then reads the status word the last call on this
+ * workspace left.  *device_status receives the MOBA_STATUS_* bits (0 = ok).
+ * Returns MOBA_OK, MOBA_EDEVICE if any bit is set, or MOBA_ELAUNCH if the
+ * stream reported a CUDA error. */
+int moba_check_status(const void* workspace, void* stream, int32_t* device_status);
+
+/* Static description of a return code. */
+const char* moba_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOBA_H_ */

@@ -62,6 +62,7 @@ __all__ = [
     "attention_backward",
     "backward_rows",
     "block_selected_by",
+    "block_index",
 ]
 
 # Largest finite bf16 value, (2 - 2^-7) * 2^127.
@@ -365,3 +366,28 @@ def block_selected_by(q_h: np.ndarray, cent_h: np.ndarray, j: int, positions: np
         beat = np.count_nonzero(sc > sj) + np.count_nonzero(sc[:j] == sj)
         out[r] = beat < topk - 1
     return out
+
+
+def block_index(sel, cu_seqlens, block_size: int, h_kv: int):
+    """Key-block-major inversion of the picks (the varlen layout of the
+    FlashMoBA Flash TopK stage 3, §"Progettazione del Kernel FlashMoBA",
+    "Tre Kernel Fusi" 1).
+
+    Returns {(kv_head, global block): sorted list of query row ids
+    t * H_q + h}, global block = (blocks of earlier sequences) + j.  Every
+    valid pick (own block included) appears once.
+    """
+    sel = np.asarray(sel)
+    T, hq, topk = sel.shape
+    g = hq // h_kv
+    seqs = _seqs(cu_seqlens)
+    out = {}
+    off = 0
+    for a, b in seqs:
+        for t in range(a, b):
+            for h in range(hq):
+                for j in sel[t, h]:
+                    if j >= 0:
+                        out.setdefault((h // g, off + int(j)), []).append(t * hq + h)
+        off += (b - a + block_size - 1) // block_size
+    return {key: sorted(v) for key, v in out.items()}

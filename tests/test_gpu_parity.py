@@ -1,0 +1,223 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded inputs.  Small cases compare every element; the full-size
+workloads compare seeded samples of rows the oracle computes one by one."""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_long_key_b200 import moba, synth
+from oracle import moba_oracle as orc
+import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+# (seqlens, h_q, h_kv, d, B, topk, conv width)
+SMALL = [
+    ((4096,), 1, 1, 64, 128, 8, 0),                 # the 4K, one-head workload in full
+    ((100, 257, 1000, 33), 4, 2, 128, 64, 4, 0),    # ragged varlen, GQA 2:1
+    ((700, 1, 15, 300), 2, 2, 64, 16, 5, 0),        # B=16, sequences of 1 and < B tokens
+    ((2048,), 2, 2, 64, 32, 32, 4),                 # small blocks + key conv width 4
+    ((1500, 0, 600), 2, 1, 128, 128, 3, 0),         # empty sequence in the middle, B=128
+    ((900,), 2, 2, 64, 32, 1, 0),                   # topk=1: block-diagonal causal
+    ((600,), 1, 1, 128, 32, 64, 0),                 # topk=64 >= n: dense causal
+    ((3000,), 8, 2, 64, 64, 16, 3),                 # GQA 4:1, conv width 3
+]
+
+
+def _ids(c):
+    return "L%s_h%dx%d_d%d_B%d_k%d_w%d" % ("-".join(map(str, c[0])), c[1], c[2], c[3], c[4], c[5], c[6])
+
+
+@pytest.fixture(scope="module")
+def dev():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    moba.lib()
+    return torch.device("cuda:0")
+
+
+def _inputs(case, seed=11):
+    seqlens, hq, hkv, d, B, topk, W = case
+    w = synth.small(seqlens, hq, hkv, d, B, topk, conv_width=W, seed=seed)
+    return w, synth.make_inputs(w)
+
+
+def _gpu(x, dev):
+    return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+
+
+@pytest.mark.parametrize("case", SMALL, ids=_ids)
+def test_forward_matches_oracle(dev, case):
+    w, x = _inputs(case)
+    g = _gpu(x, dev)
+    out, lse, sel, _ = moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], w.block_size, w.topk,
+                                    conv_w=g.get("conv_w"))
+    torch.cuda.synchronize()
+    ref = pu.oracle_forward(x, w.block_size, w.topk)
+    sel_g = sel.cpu().numpy()
+    bad = pu.selection_mismatch_rows(sel_g, ref["sel"], ref["gap"])
+    o_g, lse_g = pu.to64(out), pu.to64(lse)
+    o_ref, lse_ref = ref["o"].copy(), ref["lse"].copy()
+    if bad:   # near ties: re-check those rows under the GPU's own selection
+        o2, l2 = orc.attention(ref["q"], ref["k"], ref["v"], sel_g, ref["cu"], w.block_size, rows=bad)
+        for t, h in bad:
+            o_ref[t, h], lse_ref[t, h] = o2[t, h], l2[t, h]
+    pu.check_o_lse(o_g, lse_g, o_ref, lse_ref, _ids(case))
+
+
+@pytest.mark.parametrize("case", [c for c in SMALL if c[6] > 0] + [SMALL[1]], ids=_ids)
+def test_conv_and_centroids_match_oracle(dev, case):
+    w, x = _inputs(case)
+    g = _gpu(x, dev)
+    k_conv, cent = moba.key_conv_centroid(g["k"], g["cu_seqlens"], w.block_size, conv_w=g.get("conv_w"))
+    torch.cuda.synchronize()
+    cu = x["cu_seqlens"].numpy()
+    k = x["k"].double().numpy()
+    if w.conv_width:
+        k_ref = orc.key_conv(k, x["conv_w"].double().numpy(), cu)
+        k_g = pu.to64(k_conv)
+        diff = k_g != k_ref
+        # fp32 (GPU) vs fp64 (oracle) before the bf16 rounding: the two may
+        # straddle a rounding midpoint, never by more than one bf16 step.
+        ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(k_ref), 1e-30))) - 7)
+        assert np.all(np.abs(k_g - k_ref)[diff] <= ulp[diff] * 1.0001)
+        assert diff.mean() < 1e-3, diff.mean()
+        k = k_ref
+    cents = orc.block_centroids(k, cu, w.block_size)
+    c_g = cent.cpu().double().numpy()
+    off = 0
+    for c in cents:
+        n = c.shape[1]
+        np.testing.assert_allclose(c_g[:, off:off + n], c, rtol=1e-5, atol=1e-6)
+        off += n
+
+
+@pytest.mark.parametrize("case", SMALL[:5], ids=_ids)
+def test_block_index_matches_oracle(dev, case):
+    w, x = _inputs(case)
+    ref = pu.oracle_forward(x, w.block_size, w.topk)
+    sel = torch.tensor(ref["sel"], dtype=torch.int32, device=dev)
+    ptr, rows = moba.build_index(sel, x["cu_seqlens"].to(dev), w.h_kv, w.block_size)
+    torch.cuda.synchronize()
+    want = orc.block_index(ref["sel"], ref["cu"], w.block_size, w.h_kv)
+    ptr, rows = ptr.cpu().numpy(), rows.cpu().numpy()
+    nb = w.total_tokens // w.block_size + w.batch
+    got = {}
+    for kvh in range(w.h_kv):
+        for gb in range(nb):
+            b = kvh * nb + gb
+            if ptr[b + 1] > ptr[b]:
+                got[(kvh, gb)] = sorted(rows[ptr[b]:ptr[b + 1]].tolist())
+    assert got == want
+    assert ptr[-1] == sum(len(v) for v in want.values())
+
+
+@pytest.mark.parametrize("case", SMALL, ids=_ids)
+def test_backward_matches_oracle(dev, case):
+    w, x = _inputs(case)
+    g = _gpu(x, dev)
+    out, lse, sel, k_used = moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], w.block_size, w.topk,
+                                         conv_w=g.get("conv_w"))
+    dq, dk, dv = moba.backward(g["q"], k_used, g["v"], out, lse, g["dout"], sel, g["cu_seqlens"], w.block_size)
+    torch.cuda.synchronize()
+    ref = pu.oracle_forward(x, w.block_size, w.topk)
+    bad = pu.selection_mismatch_rows(sel.cpu().numpy(), ref["sel"], ref["gap"])
+    dq_r, dk_r, dv_r = orc.attention_backward(ref["q"], ref["k"], ref["v"], x["dout"].double().numpy(), ref["sel"],
+                                              ref["cu"], w.block_size)
+    dq_g, dk_g, dv_g = pu.to64(dq), pu.to64(dk), pu.to64(dv)
+    if bad:
+        # Rows selected differently (near ties) change dQ of that row and
+        # dK/dV of the blocks involved; leave those out.
+        keep_q = np.ones(dq_r.shape[:2], bool)
+        keep_kv = np.ones(dk_r.shape[:2], bool)
+        g_ = w.h_q // w.h_kv
+        sel_g = sel.cpu().numpy()
+        for t, h in bad:
+            keep_q[t, h] = False
+            s = int(np.searchsorted(ref["cu"], t, side="right") - 1)
+            for j in set(sel_g[t, h]) ^ set(ref["sel"][t, h]):
+                if j >= 0:
+                    a = ref["cu"][s] + j * w.block_size
+                    keep_kv[a:a + w.block_size, h // g_] = False
+        dq_r, dq_g = dq_r[keep_q], dq_g[keep_q]
+        dk_r, dk_g, dv_r, dv_g = dk_r[keep_kv], dk_g[keep_kv], dv_r[keep_kv], dv_g[keep_kv]
+    pu.check_grad(dq_g, dq_r, "dq " + _ids(case))
+    pu.check_grad(dk_g, dk_r, "dk " + _ids(case))
+    pu.check_grad(dv_g, dv_r, "dv " + _ids(case))
+
+
+def test_status_flags_bad_seqlens_without_fault(dev):
+    w, x = _inputs(((256, 256), 1, 1, 64, 32, 4, 0))
+    g = _gpu(x, dev)
+    cu = torch.tensor([0, 300, 200], dtype=torch.int32, device=dev)   # not monotone, wrong end
+    ws = moba.alloc_workspace(moba.fwd_workspace_size(moba.shape_of(g["q"], g["k"], cu, 32, 4)), dev)
+    moba.forward(g["q"], g["k"], g["v"], cu, 32, 4, workspace=ws)
+    assert moba.check_status(ws) & moba.STATUS_BAD_SEQLENS
+    ws2 = moba.alloc_workspace(moba.fwd_workspace_size(moba.shape_of(g["q"], g["k"], g["cu_seqlens"], 32, 4)), dev)
+    moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], 32, 4, workspace=ws2)
+    assert moba.check_status(ws2) == 0
+
+
+def test_status_flags_bad_sel_idx_in_backward(dev):
+    w, x = _inputs(((512,), 2, 2, 64, 32, 4, 0))
+    g = _gpu(x, dev)
+    out, lse, sel, _ = moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], 32, 4)
+    sel = sel.clone()
+    sel[3, 0, 0] = 9      # token 3 lives in block 0: block 9 is in its future
+    sel[400, 1, 0] = -7
+    shape = moba.shape_of(g["q"], g["k"], g["cu_seqlens"], 32, 4)
+    ws = moba.alloc_workspace(moba.bwd_workspace_size(shape), dev)
+    dq, dk, dv = moba.backward(g["q"], g["k"], g["v"], out, lse, g["dout"], sel, g["cu_seqlens"], 32, workspace=ws)
+    assert moba.check_status(ws) & moba.STATUS_BAD_SEL_IDX
+    assert torch.isfinite(dq.float()).all() and torch.isfinite(dk.float()).all()
+
+
+def test_repeat_calls_are_stable(dev):
+    w, x = _inputs(((1024,), 2, 2, 64, 32, 8, 0))
+    g = _gpu(x, dev)
+    a = moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], 32, 8)
+    b = moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], 32, 8)
+    assert torch.equal(a[2], b[2])
+    assert (a[0].float() - b[0].float()).abs().max().item() <= 2 ** -7
+
+
+# ------------------------------------------------------------- full sizes
+
+def _sample_rows(w, per_head, seed):
+    r = np.random.default_rng(seed)
+    rows = []
+    for h in range(w.h_q):
+        ts = r.choice(w.total_tokens, size=min(per_head, w.total_tokens), replace=False)
+        rows += [(int(t), h) for t in ts]
+    return rows
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_full_size_sampled_rows(dev, name):
+    w = synth.WORKLOADS[name]
+    x = synth.make_inputs(w)
+    g = _gpu(x, dev)
+    out, lse, sel, k_used = moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], w.block_size, w.topk,
+                                         conv_w=g.get("conv_w"))
+    dq = None
+    if w.backward:
+        dq, dk, dv = moba.backward(g["q"], k_used, g["v"], out, lse, g["dout"], sel, g["cu_seqlens"], w.block_size)
+        assert torch.isfinite(dk.float()).all() and torch.isfinite(dv.float()).all()
+    torch.cuda.synchronize()
+    rows = _sample_rows(w, 48, 7)
+    ref = pu.oracle_forward(x, w.block_size, w.topk, rows=rows)
+    sel_g = sel.cpu().numpy()
+    bad = pu.selection_mismatch_rows(sel_g, ref["sel"], ref["gap"], rows=rows)
+    o_g, lse_g = pu.to64(out), pu.to64(lse)
+    sel_use = ref["sel"].copy()
+    for t, h in bad:
+        sel_use[t, h] = sel_g[t, h]
+    o_ref, lse_ref = orc.attention(ref["q"], ref["k"], ref["v"], sel_use, ref["cu"], w.block_size, rows=rows)
+    idx = tuple(np.array(rows).T)
+    pu.check_o_lse(o_g[idx], lse_g[idx], o_ref[idx], lse_ref[idx], name)
+    for kv, hq, i, j in x["needles"]:          # planted blocks are always picked
+        assert j in sel_g[i, hq], (kv, hq, i, j)
+    if dq is not None:
+        dq_r, _ = orc.backward_rows(ref["q"], ref["k"], ref["v"], x["dout"].float().numpy(), sel_use, ref["cu"],
+                                    w.block_size, rows)
+        pu.check_grad(pu.to64(dq)[idx], dq_r, "dq " + name)

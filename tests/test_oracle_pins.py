@@ -359,3 +359,22 @@ def test_planted_needles_are_selected():
     sel, _ = orc.route(x["q"].double().numpy(), cents, x["cu_seqlens"].numpy(), w.block_size, w.topk, rows=rows)
     for (_, hq, i, j) in x["needles"]:
         assert j in sel[i, hq], (i, hq, j)
+
+
+def test_block_index_is_a_partition_of_the_picks():
+    r = _rng(15)
+    cu = [0, 30, 31, 90]
+    T, hq, hkv, d, B, topk = 90, 4, 2, 4, 8, 3
+    q = r.standard_normal((T, hq, d))
+    k = r.standard_normal((T, hkv, d))
+    sel, _ = orc.route(q, orc.block_centroids(k, cu, B), cu, B, topk)
+    idx = orc.block_index(sel, cu, B, hkv)
+    picks = [(t * hq + h, j) for t in range(T) for h in range(hq) for j in sel[t, h] if j >= 0]
+    assert sum(len(v) for v in idx.values()) == len(picks)
+    offs = [0, 4, 5]                                          # ceil(30/8), ceil(1/8)
+    for t in range(T):
+        s = 0 if t < 30 else (1 if t < 31 else 2)
+        for h in range(hq):
+            for j in sel[t, h]:
+                if j >= 0:
+                    assert t * hq + h in idx[(h // 2, offs[s] + int(j))]
