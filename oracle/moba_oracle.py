@@ -289,6 +289,8 @@ def attention_backward(q, k, v, dout, sel, cu_seqlens, block_size):
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
     for a, b in _seqs(cu_seqlens):
+        if b == a:
+            continue  # an empty sequence has no queries and no keys
         for h in range(hq):
             kv = h // g
             msk = _mask(sel, a, b, h, block_size)

@@ -6,13 +6,18 @@ Tolerances (bf16 inputs, fp32 accumulation on the GPU, fp64 oracle):
   past-block scores differ by <= 1e-3 relative; those are re-checked under
   the GPU's own selection.
 * O: max-abs <= 2e-2 and mean-abs <= 1e-3; LSE: max-abs <= 1e-3.
-* dQ/dK/dV, relative to the RMS of the oracle gradient: max-abs <= 4e-2,
-  mean-abs <= 4e-3.  Derivation: the GPU rounds P and dS to bf16 before
-  their products (relative error 2^-9 per factor, fp32 sums) and rounds the
-  result to bf16 (2^-9 = 2e-3 relative); with at most ~2 such roundings per
-  term and random signs the expected mean error is ~1.5 * 2^-9 * mean|g|
-  (~2.4e-3 rms) and the tail over 1e5..1e7 elements stays under ~5 sigma
-  of that.
+* dQ/dK/dV, element by element: |g_gpu - g_ref| <= 2e-2 * (rms(g_ref) +
+  max|g_ref row|), the row being the d values of one (token, head), and
+  mean-abs <= 4e-3 * rms(g_ref).  Derivation: each gradient element is a sum
+  of products with one factor rounded to bf16 before the MMA (P for dV, dS
+  for dQ and dK; relative error 2^-9 each, fp32 sums), so its error is
+  bounded by 2^-9 * sum|terms|, which is of the size of the largest element
+  of the same row, not of the element itself (the terms cancel: the dS of a
+  query sum to zero); the result is then rounded to bf16 (2^-9), and D_i is
+  formed from the bf16 O as in the FlashAttention-style backward.  A numpy
+  emulation with exactly those roundings reproduces the GPU values and gives
+  max |error| / (rms + row max) = 4.8e-3 and mean 1.6e-3 rms on the 4K
+  workload: the bound keeps a 4x margin over that.
 """
 from __future__ import annotations
 
@@ -23,7 +28,7 @@ from oracle import moba_oracle as orc
 
 GAP = 1e-3
 O_MAX, O_MEAN, LSE_MAX = 2e-2, 1e-3, 1e-3
-G_MAX, G_MEAN = 4e-2, 4e-3
+G_REL, G_MEAN = 2e-2, 4e-3
 
 
 def to64(t: torch.Tensor) -> np.ndarray:
@@ -56,9 +61,11 @@ def check_grad(g_gpu, g_ref, what=""):
     rms = float(np.sqrt(np.mean(g_ref ** 2))) + 1e-30
     err = np.abs(g_gpu - g_ref)
     assert np.isfinite(g_gpu).all(), what
-    assert err.max() <= G_MAX * rms, (what, "max-abs/rms", err.max() / rms)
+    rowmax = np.abs(g_ref).max(axis=-1, keepdims=True)
+    ratio = err / (G_REL * (rms + rowmax))
+    assert ratio.max() <= 1.0, (what, "max err/(2e-2*(rms+rowmax))", ratio.max(), "max-abs/rms", err.max() / rms)
     assert err.mean() <= G_MEAN * rms, (what, "mean-abs/rms", err.mean() / rms)
-    return err.max() / rms, err.mean() / rms
+    return ratio.max(), err.mean() / rms
 
 
 def oracle_forward(x: dict, B: int, topk: int, rows=None):

@@ -82,12 +82,19 @@ def test_conv_and_centroids_match_oracle(dev, case):
         assert np.all(np.abs(k_g - k_ref)[diff] <= ulp[diff] * 1.0001)
         assert diff.mean() < 1e-3, diff.mean()
         k = k_ref
+        kdiff = np.abs(k_g - k_ref)
+    else:
+        kdiff = np.zeros_like(k)
     cents = orc.block_centroids(k, cu, w.block_size)
+    # A one-step difference in a key moves its block mean by that step / n;
+    # those known key differences widen the bound of their block only.
+    slack = orc.block_centroids(kdiff, cu, w.block_size)
     c_g = cent.cpu().double().numpy()
     off = 0
-    for c in cents:
+    for c, sl in zip(cents, slack):
         n = c.shape[1]
-        np.testing.assert_allclose(c_g[:, off:off + n], c, rtol=1e-5, atol=1e-6)
+        err = np.abs(c_g[:, off:off + n] - c)
+        assert np.all(err <= 1e-6 + 1e-5 * np.abs(c) + sl * 1.0001), err.max()
         off += n
 
 

@@ -299,13 +299,14 @@ def test_backward_matches_central_finite_differences():
         np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8, err_msg=name)
 
 
-def test_backward_topk_all_equals_library_autograd():
+@pytest.mark.parametrize("cu", [[0, 30], [0, 0, 30, 30]])
+def test_backward_topk_all_equals_library_autograd(cu):
     r = _rng(12)
     T, hq, hkv, d, B = 30, 2, 1, 8, 4
     q, k, v = r.standard_normal((T, hq, d)), r.standard_normal((T, hkv, d)), r.standard_normal((T, hkv, d))
     dout = r.standard_normal((T, hq, d))
-    sel, _ = orc.route(q, orc.block_centroids(k, [0, T], B), [0, T], B, topk=100)
-    dq, dk, dv = orc.attention_backward(q, k, v, dout, sel, [0, T], B)
+    sel, _ = orc.route(q, orc.block_centroids(k, cu, B), cu, B, topk=100)
+    dq, dk, dv = orc.attention_backward(q, k, v, dout, sel, cu, B)
     tq = torch.tensor(q).permute(1, 0, 2)[None].requires_grad_()
     tk = torch.tensor(k).permute(1, 0, 2)[None].requires_grad_()
     tv = torch.tensor(v).permute(1, 0, 2)[None].requires_grad_()
