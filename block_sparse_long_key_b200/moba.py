@@ -228,6 +228,8 @@ class StageEvents:
 
     def __init__(self):
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(STAGES))]
+        for e in self.events:   # torch creates the CUDA event on its first record
+            e.record()
         self._arr = (ctypes.c_void_p * len(self.events))(*[e.cuda_event for e in self.events])
 
     def __enter__(self):

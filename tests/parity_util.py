@@ -6,18 +6,19 @@ Tolerances (bf16 inputs, fp32 accumulation on the GPU, fp64 oracle):
   past-block scores differ by <= 1e-3 relative; those are re-checked under
   the GPU's own selection.
 * O: max-abs <= 2e-2 and mean-abs <= 1e-3; LSE: max-abs <= 1e-3.
-* dQ/dK/dV, element by element: |g_gpu - g_ref| <= 2e-2 * (rms(g_ref) +
-  max|g_ref row|), the row being the d values of one (token, head), and
-  mean-abs <= 4e-3 * rms(g_ref).  Derivation: each gradient element is a sum
-  of products with one factor rounded to bf16 before the MMA (P for dV, dS
-  for dQ and dK; relative error 2^-9 each, fp32 sums), so its error is
-  bounded by 2^-9 * sum|terms|, which is of the size of the largest element
-  of the same row, not of the element itself (the terms cancel: the dS of a
-  query sum to zero); the result is then rounded to bf16 (2^-9), and D_i is
-  formed from the bf16 O as in the FlashAttention-style backward.  A numpy
-  emulation with exactly those roundings reproduces the GPU values and gives
-  max |error| / (rms + row max) = 4.8e-3 and mean 1.6e-3 rms on the 4K
-  workload: the bound keeps a 4x margin over that.
+* dQ/dK/dV, element by element: |g_gpu - g_ref| <= 4 u (s + |g_ref|) with
+  u = 2^-8 (bf16 unit roundoff) and s the first-order rounding magnitude of
+  that element (``grad_error_scales``), plus mean-abs <= 4e-3 * rms(g_ref).
+  Derivation: the GPU rounds one factor of every product to bf16 before the
+  MMAs (P for dV, dS for dQ and dK; fp32 sums), forms D_i = dO_i . O_i from
+  the bf16 output O as the FlashAttention-style backward does, and rounds the
+  results to bf16.  To first order that moves dQ_ic by at most
+  u * (sum_t |dS_it| |k_tc| + U_i sum_t P_it |k_tc|) / sqrt(d), with
+  U_i = sum_c |dO_ic O_ic| bounding the D rounding (the dS of a query sum to
+  zero, so dQ can be far smaller than its terms); dK likewise with q, and
+  dV by u * sum_i P_it |dO_ic|; each plus u |g| for the final rounding.  A
+  numpy emulation of exactly those roundings reproduces the GPU values and
+  stays within 0.45 of this bound (of 4u) on the small cases.
 """
 from __future__ import annotations
 
@@ -28,7 +29,8 @@ from oracle import moba_oracle as orc
 
 GAP = 1e-3
 O_MAX, O_MEAN, LSE_MAX = 2e-2, 1e-3, 1e-3
-G_REL, G_MEAN = 2e-2, 4e-3
+U_BF16 = 2.0 ** -8
+G_FACTOR, G_MEAN = 4.0, 4e-3
 
 
 def to64(t: torch.Tensor) -> np.ndarray:
@@ -57,15 +59,64 @@ def check_o_lse(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
     return err.max(), err.mean(), le.max()
 
 
-def check_grad(g_gpu, g_ref, what=""):
+def check_grad(g_gpu, g_ref, scale, what=""):
+    """Element-wise rounding bound (see module docstring) + mean-abs bound."""
     rms = float(np.sqrt(np.mean(g_ref ** 2))) + 1e-30
     err = np.abs(g_gpu - g_ref)
     assert np.isfinite(g_gpu).all(), what
-    rowmax = np.abs(g_ref).max(axis=-1, keepdims=True)
-    ratio = err / (G_REL * (rms + rowmax))
-    assert ratio.max() <= 1.0, (what, "max err/(2e-2*(rms+rowmax))", ratio.max(), "max-abs/rms", err.max() / rms)
+    bound = G_FACTOR * U_BF16 * (scale + np.abs(g_ref)) + 1e-6 * rms
+    ratio = err / bound
+    assert ratio.max() <= 1.0, (what, "max err / bound", ratio.max(), "max-abs/rms", err.max() / rms)
     assert err.mean() <= G_MEAN * rms, (what, "mean-abs/rms", err.mean() / rms)
     return ratio.max(), err.mean() / rms
+
+
+def grad_error_scales(q, k, v, dout, sel, cu, B, lse, o):
+    """First-order rounding magnitudes s of dQ, dK, dV (dense, small inputs).
+
+    q, k, v, dout fp64 [T, H, d]; lse, o the oracle's forward results.
+    """
+    T, hq, d = q.shape
+    g = hq // k.shape[1]
+    sc = 1.0 / np.sqrt(d)
+    sq, sk, sv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for a, b in zip(cu[:-1], cu[1:]):
+        a, b = int(a), int(b)
+        if a == b:
+            continue
+        for h in range(hq):
+            kv = h // g
+            m = orc._mask(sel, a, b, h, B)
+            qq, kk, vv, do = q[a:b, h], k[a:b, kv], v[a:b, kv], dout[a:b, h]
+            p = np.where(m, np.exp(qq @ kk.T * sc - lse[a:b, h][:, None]), 0.0)
+            D = (do * o[a:b, h]).sum(1)
+            U = np.abs(do * o[a:b, h]).sum(1)
+            ds = np.abs(p * (do @ vv.T - D[:, None]))
+            sq[a:b, h] = (ds @ np.abs(kk) + U[:, None] * (p @ np.abs(kk))) * sc
+            sk[a:b, kv] += (ds.T @ np.abs(qq) + (p * U[:, None]).T @ np.abs(qq)) * sc
+            sv[a:b, kv] += p.T @ np.abs(do)
+    return sq, sk, sv
+
+
+def row_dq_error_scale(q, k, v, dout, sel, cu, B, rows, o_rows, lse_rows):
+    """``grad_error_scales``' dQ term for individual rows (large inputs)."""
+    T, hq, d = q.shape
+    g = hq // k.shape[1]
+    sc = 1.0 / np.sqrt(d)
+    starts = np.asarray(cu)[:-1]
+    out = np.zeros((len(rows), d))
+    for r, (t, h) in enumerate(rows):
+        s = int(np.searchsorted(starts, t, side="right") - 1)
+        vis = orc.visible_tokens(sel[t, h], t, int(cu[s]), int(cu[s + 1]), B)
+        kk = np.asarray(k[vis, h // g], dtype=np.float64)
+        vv = np.asarray(v[vis, h // g], dtype=np.float64)
+        do = np.asarray(dout[t, h], dtype=np.float64)
+        p = np.exp(kk @ q[t, h] * sc - lse_rows[r])
+        D = do @ o_rows[r]
+        U = np.abs(do * o_rows[r]).sum()
+        ds = np.abs(p * (vv @ do - D))
+        out[r] = (ds @ np.abs(kk) + U * (p @ np.abs(kk))) * sc
+    return out
 
 
 def oracle_forward(x: dict, B: int, topk: int, rows=None):

@@ -128,8 +128,10 @@ def test_backward_matches_oracle(dev, case):
     torch.cuda.synchronize()
     ref = pu.oracle_forward(x, w.block_size, w.topk)
     bad = pu.selection_mismatch_rows(sel.cpu().numpy(), ref["sel"], ref["gap"])
-    dq_r, dk_r, dv_r = orc.attention_backward(ref["q"], ref["k"], ref["v"], x["dout"].double().numpy(), ref["sel"],
-                                              ref["cu"], w.block_size)
+    do64 = x["dout"].double().numpy()
+    dq_r, dk_r, dv_r = orc.attention_backward(ref["q"], ref["k"], ref["v"], do64, ref["sel"], ref["cu"], w.block_size)
+    sq, sk, sv = pu.grad_error_scales(ref["q"], ref["k"], ref["v"], do64, ref["sel"], ref["cu"], w.block_size,
+                                      ref["lse"], ref["o"])
     dq_g, dk_g, dv_g = pu.to64(dq), pu.to64(dk), pu.to64(dv)
     if bad:
         # Rows selected differently (near ties) change dQ of that row and
@@ -145,11 +147,12 @@ def test_backward_matches_oracle(dev, case):
                 if j >= 0:
                     a = ref["cu"][s] + j * w.block_size
                     keep_kv[a:a + w.block_size, h // g_] = False
-        dq_r, dq_g = dq_r[keep_q], dq_g[keep_q]
+        dq_r, dq_g, sq = dq_r[keep_q], dq_g[keep_q], sq[keep_q]
         dk_r, dk_g, dv_r, dv_g = dk_r[keep_kv], dk_g[keep_kv], dv_r[keep_kv], dv_g[keep_kv]
-    pu.check_grad(dq_g, dq_r, "dq " + _ids(case))
-    pu.check_grad(dk_g, dk_r, "dk " + _ids(case))
-    pu.check_grad(dv_g, dv_r, "dv " + _ids(case))
+        sk, sv = sk[keep_kv], sv[keep_kv]
+    pu.check_grad(dq_g, dq_r, sq, "dq " + _ids(case))
+    pu.check_grad(dk_g, dk_r, sk, "dk " + _ids(case))
+    pu.check_grad(dv_g, dv_r, sv, "dv " + _ids(case))
 
 
 def test_status_flags_bad_seqlens_without_fault(dev):
@@ -225,6 +228,8 @@ def test_full_size_sampled_rows(dev, name):
     for kv, hq, i, j in x["needles"]:          # planted blocks are always picked
         assert j in sel_g[i, hq], (kv, hq, i, j)
     if dq is not None:
-        dq_r, _ = orc.backward_rows(ref["q"], ref["k"], ref["v"], x["dout"].float().numpy(), sel_use, ref["cu"],
-                                    w.block_size, rows)
-        pu.check_grad(pu.to64(dq)[idx], dq_r, "dq " + name)
+        do32 = x["dout"].float().numpy()
+        dq_r, _ = orc.backward_rows(ref["q"], ref["k"], ref["v"], do32, sel_use, ref["cu"], w.block_size, rows)
+        s_r = pu.row_dq_error_scale(ref["q"], ref["k"], ref["v"], do32, sel_use, ref["cu"], w.block_size, rows,
+                                    o_ref[idx], lse_ref[idx])
+        pu.check_grad(pu.to64(dq)[idx], dq_r, s_r, "dq " + name)
