@@ -151,6 +151,37 @@ int moba_build_index(const int32_t* sel_idx, const int32_t* cu_seqlens, const mo
                      void* stream);
 
 /*
+ * Allocation-free moba_build_index.  The paper has no counterpart: this entry
+ * point exists for callers that cannot provide device scratch memory, such
+ * as code running inside a host framework that owns all device memory and
+ * forbids side allocations, or latency-critical paths that must not call
+ * cudaMalloc because it can synchronise the device.
+ *
+ * Same inputs, outputs and results as moba_build_index, without the
+ * workspace: its scratch lives in a static device array of
+ * MOBA_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that
+ * loads the library keeps until the process exits.  The call allocates and
+ * frees nothing.
+ *
+ *  - Runs on the current device; `stream` must belong to it.  The first call
+ *    on each device looks up the array's device address (cudaGetSymbolAddress)
+ *    and caches it; make that first call before any stream capture.
+ *  - Every call on a device shares the one array, and the array keeps what the
+ *    last call left in it (this call clears what must start at zero).  Calls
+ *    whose work overlaps on the GPU (other streams, other host threads) race
+ *    on it and give wrong results: serialise them.
+ *  - The scratch holds 4 * (h_kv * (T / B + batch)) * 2 bytes of counters and
+ *    cursors plus 3 * 4 * (batch + 1) bytes of sequence plan (each part rounded
+ *    up to 256 bytes, plus 256); a shape that needs more than
+ *    MOBA_NOALLOC_SCRATCH_BYTES returns MOBA_EWORKSPACE and launches nothing.
+ *  - Device-side input errors (bad cu_seqlens or sel_idx) are skipped, as in
+ *    moba_build_index; the status word is not readable from outside here.
+ */
+#define MOBA_NOALLOC_SCRATCH_BYTES (8u << 20)
+int moba_build_index_noalloc(const int32_t* sel_idx, const int32_t* cu_seqlens, const moba_shape* shape,
+                             int32_t* blk_ptr, int32_t* blk_rows, void* stream);
+
+/*
  * MoBA backward with the selection held fixed ("Optimizing Mixture of Block
  * Attention", section "Progettazione del Kernel FlashMoBA", "Tre Kernel
  * Fusi" 3: recompute per key block, dQ by atomic accumulation in fp32).
