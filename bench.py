@@ -412,6 +412,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(synth.WORKLOADS), default=synth.HEADLINE)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the KV head count (query heads scale with it); for small profiling runs")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=1500, help="oracle rows per CPU-baseline step")
@@ -419,6 +421,13 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
+    if args.heads:
+        import dataclasses
+        w = synth.WORKLOADS[args.workload]
+        g = w.h_q // w.h_kv
+        name = "%s_kvheads%d" % (w.name, args.heads)
+        synth.WORKLOADS[name] = dataclasses.replace(w, name=name, h_kv=args.heads, h_q=args.heads * g)
+        args.workload = name
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -12,7 +12,8 @@ namespace moba {
 enum : int32_t {
   kStatusBadSeqlens = 1 << 0,   // cu_seqlens not monotone / not ending at T
   kStatusBadSelIdx = 1 << 1,    // sel_idx entry outside [-1, own block]
-  kStatusIndexOverflow = 1 << 2 // CSR fill ran past its bucket
+  kStatusIndexOverflow = 1 << 2, // CSR fill ran past its bucket
+  kStatusTimeout = 1 << 3        // a bounded wait on the tensor cores gave up
 };
 
 __device__ __forceinline__ void set_status(int32_t* status, int32_t bit) {

@@ -13,7 +13,7 @@ namespace moba {
 typedef __nv_bfloat16 bf16;
 
 // Query rows per routing tile.
-constexpr int kRouteTile = 64;
+constexpr int kRouteTile = 128;
 
 struct SeqPlan {
   const int32_t* cu;        // sanitised cu_seqlens [batch + 1]
@@ -35,7 +35,7 @@ cudaError_t launch_conv_centroid(const bf16* k, const float* conv_w, int conv_wi
 cudaError_t launch_route(const bf16* q, const bf16* k, const bf16* cent_hi, const bf16* cent_lo,
                          const SeqPlan& p, int h_q, int h_kv, int d, int block_size, int topk,
                          int32_t* sel_idx, float* mref, int32_t* flag, float* lacc, float* oacc,
-                         cudaStream_t st);
+                         int32_t* status, cudaStream_t st);
 
 cudaError_t launch_build_index(const int32_t* sel_idx, const SeqPlan& p, int h_q, int h_kv,
                                int block_size, int topk, int32_t* cnt, int32_t* ptr, int32_t* cursor,

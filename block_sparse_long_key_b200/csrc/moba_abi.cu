@@ -242,7 +242,7 @@ int moba_forward(const void* q, const void* k, const void* v, const int32_t* cu_
   STAGE_END(MOBA_STAGE_FWD_CENTROID);
   STAGE_BEGIN(MOBA_STAGE_FWD_ROUTE);
   MOBA_TRY(moba::launch_route(kq, kk, b.hi, b.lo, plan, hq, hkv, d, B, topk, sel_idx, b.mref, b.flag, b.lacc, b.oacc,
-                              st));
+                              b.plan.status, st));
   STAGE_END(MOBA_STAGE_FWD_ROUTE);
   STAGE_BEGIN(MOBA_STAGE_FWD_INDEX);
   MOBA_TRY(moba::launch_build_index(sel_idx, plan, hq, hkv, B, topk, b.cnt, b.ptr, b.cursor, b.rows,

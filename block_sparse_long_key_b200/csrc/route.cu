@@ -1,82 +1,92 @@
-// Router: block scores on tensor cores and per-query top-k in registers.
+// Router: block scores on the tcgen05 tensor cores, per-query top-k on the
+// CUDA cores.
 //
 // "Optimizing Mixture of Block Attention", §"Architettura del Modello
 // Statistico" 1 (router score s_j = q^T k~_j) and §"Definizione del Compito"
 // (each query keeps the top-k blocks, k << n); the FlashMoBA "Flash TopK"
-// stage 2 (§"Progettazione del Kernel FlashMoBA", "Tre Kernel Fusi" 1)
-// computes these scores tile by tile without materialising the N x n matrix;
-// this kernel does the same on sm_100a.
+// stage 2 (§"Progettazione del Kernel FlashMoBA", "Tre Kernel Fusi" 1) scores
+// tile by tile without materialising the N x n matrix; so does this kernel.
 //
 // Selection rule: a query at local position p (block b = p / B) scores the
 // earlier blocks j < b only, keeps the topk-1 best (exact ties: lower j
 // wins) and always keeps its own block b.  sel_idx rows are sorted
 // ascending and padded with -1.
 //
-// A CTA owns 64 consecutive queries of one sequence and one query head.
-// Centroid tiles of 64 blocks stream through shared memory (cp.async, double
-// buffered); each warp forms a 16 x 64 score tile with bf16 mma (fp32
-// accumulate) as q.c_hi + q.c_lo, which carries ~16 mantissa bits of the fp32
-// centroid.  Two threads per query row then fold the tile into a running
-// top-(k-1) list held in registers as 64-bit keys (order-preserving float
-// bits << 32 | ~index): one compare per score, an insertion pass only when a
-// score beats the current threshold.
+// One CTA owns 128 consecutive queries of one sequence and one query head.
+// Their Q tile and a stream of centroid chunks (NC blocks each, double
+// buffered, cp.async into 128-byte-swizzled K-major shared memory) feed
+// tcgen05.mma (M = 128 queries, N = NC blocks, bf16 in, fp32 accumulate into
+// tensor memory, double buffered): one thread issues q.c_hi + q.c_lo, which
+// carries ~16 mantissa bits of the fp32 centroid, while the CTA's 128 threads
+// select on the previous chunk.  Thread t owns query row t, which is TMEM lane
+// t: tcgen05.ld hands it that row's NC scores in registers.  Scores above the
+// thread's running threshold (the worst of its current k-1 best) go to a
+// small per-thread candidate buffer in shared memory; the whole warp flushes
+// the buffers together.  The k-1 kept entries sit unsorted in shared memory
+// ([slot][thread], so every access is bank-conflict free) in groups of 8
+// whose worst entries are tracked in registers: admitting a candidate
+// overwrites the worst slot and rescans one group plus the group minima, a
+// fixed 8 + k/8 steps whatever the data (a sorted list would shift up to k-1
+// entries, and a warp pays for its slowest lane).  Order: higher score first,
+// equal scores by lower block index.
 //
 // Side outputs for the forward: mref = a lower bound of the query's largest
 // attention logit, max(best kept score, q_i.k_i) / sqrt(d) (a block mean never
-// exceeds the block max), used as the fixed softmax reference; the query's
-// accumulator row (oacc, lacc, flag) is zeroed here.
+// exceeds the block max), the fixed softmax reference of the forward; the
+// query's accumulator row (oacc, lacc, flag) is zeroed here.
 #include "common.cuh"
 #include "launch.h"
+#include "tc.cuh"
 
 namespace moba {
 namespace {
 
-constexpr int kTM = kRouteTile;  // query rows per CTA
-constexpr int kNC = 64;          // blocks per centroid chunk
+constexpr int kTM = kRouteTile;  // query rows per CTA (= TMEM lanes)
 constexpr int kThreads = 128;
-constexpr uint64_t kSentinel = ~0ull;
+constexpr int kGroup = 8;        // kept-list slots per group
+constexpr uint32_t kFull = 0xffffffffu;
 
-__device__ __forceinline__ uint32_t order_bits(float v) {
-  uint32_t u = __float_as_uint(v);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float from_order_bits(uint32_t u) {
-  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
-}
-__device__ __forceinline__ uint64_t make_key(float v, int j) {
-  return ((uint64_t)order_bits(v) << 32) | (uint64_t)(0xffffffffu - (uint32_t)j);
-}
-
-template <int LISTN>
-__device__ __forceinline__ void list_insert(uint64_t (&L)[LISTN], uint64_t key) {
-  if (key <= L[LISTN - 1]) return;
-  uint64_t x = key;
-#pragma unroll
-  for (int m = 0; m < LISTN; ++m) {
-    const uint64_t a = L[m];
-    L[m] = a > x ? a : x;
-    x = a > x ? x : a;
-  }
-}
-
-template <int D>
-struct RouteSmem {
-  bf16 q[kTM][D + 8];
-  bf16 ch[2][kNC][D + 8];
-  bf16 cl[2][kNC][D + 8];
-  float s[kTM][kNC + 2];
+template <int D, int NC, int LISTN>
+struct RouteLayout {
+  static constexpr int kBuf = D == 64 ? 16 : 12;          // candidate buffer slots per thread
+  static constexpr int KB = D / 64;                       // 128-byte K blocks
+  static constexpr uint32_t Q_OFF = 0;
+  static constexpr uint32_t Q_REGION = kTM * 128;
+  static constexpr uint32_t C_OFF = Q_OFF + KB * Q_REGION;
+  static constexpr uint32_t C_REGION = NC * 128;
+  static constexpr uint32_t C_MAT = KB * C_REGION;       // hi or lo of one chunk
+  static constexpr uint32_t C_BUF = 2 * C_MAT;           // hi + lo
+  static constexpr uint32_t LV_OFF = C_OFF + 2 * C_BUF;
+  static constexpr uint32_t LI_OFF = LV_OFF + LISTN * kThreads * 4;
+  static constexpr uint32_t BV_OFF = LI_OFF + LISTN * kThreads * 4;
+  static constexpr uint32_t BI_OFF = BV_OFF + kBuf * kThreads * 4;
+  static constexpr uint32_t MB_OFF = BI_OFF + kBuf * kThreads * 4;
+  static_assert(LISTN % kGroup == 0, "kept list is whole groups");
+  static constexpr uint32_t HOLD_OFF = MB_OFF + 16;
+  static constexpr uint32_t FLAG_OFF = HOLD_OFF + 4;
+  static constexpr uint32_t BYTES = FLAG_OFF + 12;
+  static constexpr uint32_t TMEM_COLS = 2 * NC;
+  static_assert(C_REGION % 1024 == 0 && Q_REGION % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
+  static_assert(TMEM_COLS >= 32 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation is a power of two");
 };
 
-template <int D, int LISTN>
+template <int D, int NC, int LISTN>
 __global__ void __launch_bounds__(kThreads)
 route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ cent_hi,
              const bf16* __restrict__ cent_lo, const int32_t* __restrict__ cu,
              const int32_t* __restrict__ blk_off, const int32_t* __restrict__ tile_off, int batch,
              int nb_max, int h_q, int h_kv, int block_size, int topk, int32_t* __restrict__ sel_idx,
              float* __restrict__ mref, int32_t* __restrict__ flag, float* __restrict__ lacc,
-             float* __restrict__ oacc) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  RouteSmem<D>& sm = *reinterpret_cast<RouteSmem<D>*>(smem_raw);
+             float* __restrict__ oacc, int32_t* __restrict__ status) {
+  using Ly = RouteLayout<D, NC, LISTN>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(sm);
+  float* lv = reinterpret_cast<float*>(sm + Ly::LV_OFF);
+  int32_t* li = reinterpret_cast<int32_t*>(sm + Ly::LI_OFF);
+  float* bv = reinterpret_cast<float*>(sm + Ly::BV_OFF);
+  int32_t* bi = reinterpret_cast<int32_t*>(sm + Ly::BI_OFF);
+  const uint32_t mbar0 = sbase + Ly::MB_OFF;
 
   const int ntiles = __ldg(tile_off + batch);
   const int tile = ntiles - 1 - (int)blockIdx.x;  // longest rows first
@@ -90,30 +100,88 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   const int nrows = min(kTM, L - p0);
   const int t0 = seq0 + p0;
   const int cbase = __ldg(blk_off + s);
-  const int nscan = (p0 + nrows - 1) / block_size;  // blocks any row may score
-  const int nchunks = (nscan + kNC - 1) / kNC;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int k1 = topk - 1;
+  const int nscan = k1 > 0 ? (p0 + nrows - 1) / block_size : 0;  // blocks any row may score
+  const int nchunks = (nscan + NC - 1) / NC;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const size_t qstride = (size_t)h_q * D;
 
-  // Q tile (zero rows past the sequence end).
+  // ---- loads: Q tile, centroid chunks (hi, lo), all into SW128 K-major layout
   for (int i = tid; i < kTM * (D / 8); i += kThreads) {
-    const int r = i / (D / 8), c = i % (D / 8);
+    const int r = i / (D / 8), cc = i % (D / 8);
     const bool ok = r < nrows;
-    cp_async16_zfill(&sm.q[r][c * 8], q + (ok ? (size_t)(t0 + r) * qstride + (size_t)h * D + c * 8 : 0), ok);
+    const size_t src = ok ? (size_t)(t0 + r) * qstride + (size_t)h * D + cc * 8 : 0;
+    cp_async16_zfill(sm + Ly::Q_OFF + (cc >> 3) * Ly::Q_REGION + tc::sw128_offset(r, cc & 7), q + src, ok);
   }
+  const size_t head0 = ((size_t)kvh * nb_max + cbase) * D;
   auto load_chunk = [&](int c, int buf) {
-    const size_t head0 = ((size_t)kvh * nb_max + cbase) * D;
-    for (int i = tid; i < kNC * (D / 8); i += kThreads) {
-      const int n = i / (D / 8), cc = i % (D / 8);
-      const int jb = c * kNC + n;
+    for (int i = tid; i < 2 * NC * (D / 8); i += kThreads) {
+      const int m = i / (NC * (D / 8));
+      const int rem = i % (NC * (D / 8));
+      const int n = rem / (D / 8), cc = rem % (D / 8);
+      const int jb = c * NC + n;
       const bool ok = jb < nscan;
-      const size_t off = ok ? head0 + (size_t)jb * D + cc * 8 : 0;
-      cp_async16_zfill(&sm.ch[buf][n][cc * 8], cent_hi + off, ok);
-      cp_async16_zfill(&sm.cl[buf][n][cc * 8], cent_lo + off, ok);
+      const size_t src = ok ? head0 + (size_t)jb * D + cc * 8 : 0;
+      unsigned char* dst = sm + Ly::C_OFF + buf * Ly::C_BUF + m * Ly::C_MAT + (cc >> 3) * Ly::C_REGION +
+                           tc::sw128_offset(n, cc & 7);
+      cp_async16_zfill(dst, (m ? cent_lo : cent_hi) + src, ok);
     }
   };
   if (nchunks > 0) load_chunk(0, 0);
   cp_async_commit();
+  if (nchunks > 1) load_chunk(1, 1);
+  cp_async_commit();
+
+  // ---- per-thread selection state; TMEM + barriers
+  const bool row_ok = tid < nrows;
+  const int my_b = row_ok ? (p0 + tid) / block_size : 0;
+  // Kept list: k1 live slots start as (-inf, INT_MAX) placeholders, the padding
+  // slots up to LISTN hold +inf and are never evicted.
+  constexpr int NG = LISTN / kGroup;
+  float gv[NG];
+  int gj[NG], gs[NG];
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    gv[g] = INFINITY;
+    gj[g] = -1;
+    gs[g] = g * kGroup;
+#pragma unroll
+    for (int e = 0; e < kGroup; ++e) {
+      const int sl = g * kGroup + e;
+      const bool live = sl < k1;
+      lv[sl * kThreads + tid] = live ? -INFINITY : INFINITY;
+      li[sl * kThreads + tid] = live ? 0x7fffffff : -1;
+      if (live && gv[g] == INFINITY) {
+        gv[g] = -INFINITY;
+        gj[g] = 0x7fffffff;
+        gs[g] = sl;
+      }
+    }
+  }
+  // worst kept entry (the threshold) = worst of the group minima
+  float tau = -INFINITY;
+  int tau_j = 0x7fffffff, tau_s = 0;
+  auto worse = [](float av, int aj, float bv, int bj) { return av < bv || (av == bv && aj > bj); };
+  auto refresh_tau = [&]() {
+    tau = gv[0];
+    tau_j = gj[0];
+    tau_s = gs[0];
+#pragma unroll
+    for (int g = 1; g < NG; ++g)
+      if (worse(gv[g], gj[g], tau, tau_j)) {
+        tau = gv[g];
+        tau_j = gj[g];
+        tau_s = gs[g];
+      }
+  };
+  refresh_tau();
+  int cnt = 0;
+  if (tid == 0) {
+    tc::mbar_init(mbar0, 1);
+    tc::mbar_init(mbar0 + 8, 1);
+    tc::mbar_init_fence();
+  }
+  if (nchunks > 0 && warp == 0) tc::tmem_alloc(sbase + Ly::HOLD_OFF, Ly::TMEM_COLS);
 
   // Zero this tile's accumulator rows while the loads fly.
   for (int i = tid; i < nrows * (D / 4); i += kThreads) {
@@ -121,118 +189,179 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
     const size_t row = (size_t)(t0 + r) * h_q + h;
     reinterpret_cast<float4*>(oacc + row * D)[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
+  constexpr uint32_t idesc = tc::idesc_bf16_f32(kTM, NC);
 
-  // Per-thread running list: row r = tid / 2, column parity = tid % 2.
-  const int my_row = tid >> 1, parity = tid & 1;
-  const int my_b = (p0 + my_row) / block_size;
-  const int k1 = topk - 1;
-  uint64_t list[LISTN];
+  // Admit (x, j), x > tau: overwrite the worst slot, rescan its group, then
+  // the group minima.  Candidates arrive in ascending j, so a score equal to
+  // the threshold never displaces it (lower index wins ties).
+  auto admit = [&](float x, int j) {
+    const int s0 = tau_s;
+    lv[s0 * kThreads + tid] = x;
+    li[s0 * kThreads + tid] = j;
+    const int g0 = s0 / kGroup;
+    float mv = INFINITY;
+    int mj = -1, ms = g0 * kGroup;
 #pragma unroll
-  for (int m = 0; m < LISTN; ++m) list[m] = m < LISTN - k1 ? kSentinel : 0ull;
+    for (int e = 0; e < kGroup; ++e) {
+      const int sl = g0 * kGroup + e;
+      const float v = lv[sl * kThreads + tid];
+      const int jj = li[sl * kThreads + tid];
+      if (worse(v, jj, mv, mj)) {
+        mv = v;
+        mj = jj;
+        ms = sl;
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < NG; ++g)
+      if (g == g0) {
+        gv[g] = mv;
+        gj[g] = mj;
+        gs[g] = ms;
+      }
+    refresh_tau();
+  };
+  auto flush = [&]() {
+    for (int e = 0; e < cnt; ++e) {
+      const float x = bv[e * kThreads + tid];
+      if (x > tau) admit(x, bi[e * kThreads + tid]);
+    }
+    cnt = 0;
+  };
 
-  uint32_t qa[D / 16][4];
-  for (int c = 0; c < nchunks; ++c) {
+  auto select_chunk = [&](int c, int buf) {
+    uint32_t v[NC];
+    const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(buf * NC);
+#pragma unroll
+    for (int hf = 0; hf < NC / 32; ++hf)
+      tc::tmem_ld32(taddr + hf * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[hf * 32]));
+    tc::tmem_ld_wait();
+    const int jbase = c * NC;
+#pragma unroll
+    for (int g = 0; g < NC / 8; ++g) {
+      if (__any_sync(kFull, cnt > Ly::kBuf - 8)) flush();  // room for the next 8 columns
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int col = g * 8 + e;
+        const float x = __uint_as_float(v[col]);
+        const int j = jbase + col;
+        if (j < my_b && x > tau) {
+          bv[cnt * kThreads + tid] = x;
+          bi[cnt * kThreads + tid] = j;
+          ++cnt;
+        }
+      }
+    }
+    if (__any_sync(kFull, cnt > 0)) flush();
+  };
+
+  // All waits are decided block-wide (__syncthreads_and), so every thread
+  // takes the same path if a tensor-core completion never arrives.
+  bool ok = true;
+  for (int c = 0; c < nchunks && ok; ++c) {
     const int buf = c & 1;
-    if (c + 1 < nchunks) load_chunk(c + 1, buf ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();
+    if (c == 0 && nchunks > 1) cp_async_wait<1>(); else cp_async_wait<0>();
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
     __syncthreads();
-    if (c == 0) {
+    if (tid == 0) {
+      tc::fence_after_sync();
+      const uint32_t d_tmem = tmem + (uint32_t)(buf * NC);
+      const uint32_t qa = sbase + Ly::Q_OFF;
+      const uint32_t ca = sbase + Ly::C_OFF + buf * Ly::C_BUF;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        const int r = warp * 16 + (lane & 15), col = kk * 16 + (lane >> 4) * 8;
-        ldsm_x4(qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], &sm.q[r][col]);
+        const uint32_t koff = (kk & 3) * 32;  // 16 bf16 per K step inside a 128-byte row
+        const uint64_t a = tc::sw128_desc(qa + (kk >> 2) * Ly::Q_REGION + koff);
+        tc::mma_bf16_ss(d_tmem, a, tc::sw128_desc(ca + (kk >> 2) * Ly::C_REGION + koff), idesc, kk > 0);
       }
-    }
-    float acc[kNC / 8][4];
-#pragma unroll
-    for (int nt = 0; nt < kNC / 8; ++nt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-#pragma unroll
-    for (int nt2 = 0; nt2 < kNC / 16; ++nt2) {
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        const int n = nt2 * 16 + (lane & 7) + ((lane >> 4) << 3);
-        const int col = kk * 16 + ((lane >> 3) & 1) * 8;
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(b0, b1, b2, b3, &sm.ch[buf][n][col]);
-        mma_bf16(acc[2 * nt2], qa[kk], b0, b1);
-        mma_bf16(acc[2 * nt2 + 1], qa[kk], b2, b3);
-        ldsm_x4(b0, b1, b2, b3, &sm.cl[buf][n][col]);
-        mma_bf16(acc[2 * nt2], qa[kk], b0, b1);
-        mma_bf16(acc[2 * nt2 + 1], qa[kk], b2, b3);
+        const uint32_t koff = (kk & 3) * 32;
+        const uint64_t a = tc::sw128_desc(qa + (kk >> 2) * Ly::Q_REGION + koff);
+        tc::mma_bf16_ss(d_tmem, a, tc::sw128_desc(ca + Ly::C_MAT + (kk >> 2) * Ly::C_REGION + koff), idesc, 1u);
       }
+      tc::mma_commit(mbar0 + 8 * buf);
     }
-#pragma unroll
-    for (int nt = 0; nt < kNC / 8; ++nt) {
-      const int r = warp * 16 + (lane >> 2), col = nt * 8 + (lane & 3) * 2;
-      *reinterpret_cast<float2*>(&sm.s[r][col]) = make_float2(acc[nt][0], acc[nt][1]);
-      *reinterpret_cast<float2*>(&sm.s[r + 8][col]) = make_float2(acc[nt][2], acc[nt][3]);
-    }
-    __syncthreads();
-    if (k1 > 0 && my_row < nrows) {
-      const int jlim = min(my_b - c * kNC, kNC);  // columns [0, jlim) are past blocks of my row
-#pragma unroll 8
-      for (int i = 0; i < kNC / 2; ++i) {
-        const int col = 2 * i + parity;
-        if (col < jlim) list_insert<LISTN>(list, make_key(sm.s[my_row][col], c * kNC + col));
+    if (c >= 1) {
+      const int pc = c - 1;
+      const bool got = tc::mbar_wait(mbar0 + 8 * (pc & 1), (pc >> 1) & 1);
+      if (!__syncthreads_and(got)) {
+        ok = false;
+        break;
       }
+      if (c + 1 < nchunks) load_chunk(c + 1, (c + 1) & 1);
+      cp_async_commit();
+      tc::fence_after_sync();
+      select_chunk(pc, pc & 1);
+      tc::fence_before_sync();
+    }
+  }
+  if (nchunks > 0 && ok) {
+    const int pc = nchunks - 1;
+    const bool got = tc::mbar_wait(mbar0 + 8 * (pc & 1), (pc >> 1) & 1);
+    if (__syncthreads_and(got)) {
+      tc::fence_after_sync();
+      select_chunk(pc, pc & 1);
+    } else {
+      ok = false;
     }
   }
   cp_async_wait<0>();
+  tc::fence_before_sync();
   __syncthreads();
-
-  // Merge the two half lists of each row (odd threads hand theirs over).
-  // ch and cl are adjacent: together they hold the [kTM][LISTN] hand-over.
-  uint64_t* xfer = reinterpret_cast<uint64_t*>(&sm.ch[0][0][0]);
-  static_assert(sizeof(sm.ch) + sizeof(sm.cl) >= sizeof(uint64_t) * kTM * LISTN, "merge buffer");
-  if (parity == 1) {
-#pragma unroll
-    for (int m = 0; m < LISTN; ++m) xfer[my_row * LISTN + m] = list[m];
+  if (!ok) {
+    // A tensor-core completion never arrived: record it, give the MMAs in
+    // flight a bounded chance to drain, release TMEM, leave outputs unwritten.
+    if (tid == 0) set_status(status, kStatusTimeout);
+    tc::mbar_wait(mbar0 + 8 * ((nchunks - 1) & 1), ((nchunks - 1) >> 1) & 1, 100000000ull);
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, Ly::TMEM_COLS);
+    return;
   }
-  __syncthreads();
-  int32_t* idx_buf = reinterpret_cast<int32_t*>(&sm.s[0][0]);  // [kTM][LISTN + 1]
-  static_assert(sizeof(sm.s) >= sizeof(int32_t) * kTM * (LISTN + 1), "index buffer");
-  if (parity == 0 && my_row < nrows) {
-    for (int m = 0; m < LISTN; ++m) {
-      const uint64_t key = xfer[my_row * LISTN + m];
-      if (key != kSentinel && key != 0ull) list_insert<LISTN>(list, key);
-    }
-    // Kept past blocks (unordered), best score for the softmax reference.
-    int* mine = idx_buf + my_row * (LISTN + 1);
-    int cnt = 0;
+  if (nchunks > 0 && warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, Ly::TMEM_COLS);
+  }
+
+  if (row_ok) {
+    // Kept past blocks: compact the live slots holding a real score, note the
+    // best score, sort the block indices ascending.
+    int kept = 0;
     float best = -INFINITY;
-#pragma unroll
-    for (int m = 0; m < LISTN; ++m) {
-      const uint64_t key = list[m];
-      if (key != kSentinel && key != 0ull) {
-        mine[cnt++] = (int)(0xffffffffu - (uint32_t)(key & 0xffffffffu));
-        best = fmaxf(best, from_order_bits((uint32_t)(key >> 32)));
+    for (int sl = 0; sl < k1; ++sl) {
+      const float v = lv[sl * kThreads + tid];
+      if (v > -INFINITY) {
+        best = fmaxf(best, v);
+        li[kept * kThreads + tid] = li[sl * kThreads + tid];
+        ++kept;
       }
     }
-    // Insertion sort ascending (at most 63 entries, once per query).
-    for (int a = 1; a < cnt; ++a) {
-      const int x = mine[a];
+    for (int a = 1; a < kept; ++a) {
+      const int x = li[a * kThreads + tid];
       int b2 = a - 1;
-      while (b2 >= 0 && mine[b2] > x) {
-        mine[b2 + 1] = mine[b2];
+      while (b2 >= 0 && li[b2 * kThreads + tid] > x) {
+        li[(b2 + 1) * kThreads + tid] = li[b2 * kThreads + tid];
         --b2;
       }
-      mine[b2 + 1] = x;
+      li[(b2 + 1) * kThreads + tid] = x;
     }
-    const int t = t0 + my_row;
+    const int t = t0 + tid;
     const size_t row = (size_t)t * h_q + h;
     int32_t* out = sel_idx + row * topk;
-    for (int m = 0; m < topk; ++m) out[m] = m < cnt ? mine[m] : (m == cnt ? my_b : -1);
-    // q_i . k_i for the diagonal logit (own key is always visible).
+    for (int m = 0; m < topk; ++m) out[m] = m < kept ? li[m * kThreads + tid] : (m == kept ? my_b : -1);
+    const bf16* qrow = q + (size_t)t * qstride + (size_t)h * D;
     const bf16* krow = k + ((size_t)t * h_kv + kvh) * D;
     float dot = 0.f;
 #pragma unroll 4
     for (int c8 = 0; c8 < D / 8; ++c8) {
       float fk[8], fq[8];
       bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(krow + c8 * 8)), fk);
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(&sm.q[my_row][c8 * 8]), fq);
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow + c8 * 8)), fq);
 #pragma unroll
       for (int i = 0; i < 8; ++i) dot = fmaf(fq[i], fk[i], dot);
     }
@@ -242,19 +371,19 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   }
 }
 
-template <int D, int LISTN>
+template <int D, int NC, int LISTN>
 cudaError_t launch_route_t(const bf16* q, const bf16* k, const bf16* hi, const bf16* lo, const SeqPlan& p,
                            int h_q, int h_kv, int block_size, int topk, int32_t* sel, float* mref,
-                           int32_t* flag, float* lacc, float* oacc, cudaStream_t st) {
-  const size_t smem = sizeof(RouteSmem<D>);
-  auto kern = route_kernel<D, LISTN>;
+                           int32_t* flag, float* lacc, float* oacc, int32_t* status, cudaStream_t st) {
+  const size_t smem = RouteLayout<D, NC, LISTN>::BYTES + 1024;
+  auto kern = route_kernel<D, NC, LISTN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int max_tiles = p.total_tokens / kTM + p.batch;
   if (max_tiles == 0) return cudaSuccess;
   dim3 grid(max_tiles, h_q);
   kern<<<grid, kThreads, smem, st>>>(q, k, hi, lo, p.cu, p.blk_off, p.tile_off, p.batch, p.nb_max, h_q, h_kv,
-                                     block_size, topk, sel, mref, flag, lacc, oacc);
+                                     block_size, topk, sel, mref, flag, lacc, oacc, status);
   return cudaGetLastError();
 }
 
@@ -262,20 +391,16 @@ cudaError_t launch_route_t(const bf16* q, const bf16* k, const bf16* hi, const b
 
 cudaError_t launch_route(const bf16* q, const bf16* k, const bf16* hi, const bf16* lo, const SeqPlan& p,
                          int h_q, int h_kv, int d, int block_size, int topk, int32_t* sel, float* mref,
-                         int32_t* flag, float* lacc, float* oacc, cudaStream_t st) {
+                         int32_t* flag, float* lacc, float* oacc, int32_t* status, cudaStream_t st) {
   const int k1 = topk - 1;
-#define MOBA_ROUTE(DD, LN) \
-  return launch_route_t<DD, LN>(q, k, hi, lo, p, h_q, h_kv, block_size, topk, sel, mref, flag, lacc, oacc, st)
+#define MOBA_ROUTE(DD, NCC, LN) \
+  return launch_route_t<DD, NCC, LN>(q, k, hi, lo, p, h_q, h_kv, block_size, topk, sel, mref, flag, lacc, oacc, status, st)
   if (d == 64) {
-    if (k1 <= 8) MOBA_ROUTE(64, 8);
-    if (k1 <= 16) MOBA_ROUTE(64, 16);
-    if (k1 <= 32) MOBA_ROUTE(64, 32);
-    MOBA_ROUTE(64, 64);
+    if (k1 <= 32) MOBA_ROUTE(64, 64, 32);
+    MOBA_ROUTE(64, 64, 64);
   } else {
-    if (k1 <= 8) MOBA_ROUTE(128, 8);
-    if (k1 <= 16) MOBA_ROUTE(128, 16);
-    if (k1 <= 32) MOBA_ROUTE(128, 32);
-    MOBA_ROUTE(128, 64);
+    if (k1 <= 32) MOBA_ROUTE(128, 32, 32);
+    MOBA_ROUTE(128, 32, 64);
   }
 #undef MOBA_ROUTE
 }

@@ -73,6 +73,7 @@ typedef struct moba_shape {
 #define MOBA_STATUS_BAD_SEQLENS 1 /* cu_seqlens not monotone or not ending at T */
 #define MOBA_STATUS_BAD_SEL_IDX 2 /* a sel_idx entry outside [-1, own block]; skipped */
 #define MOBA_STATUS_INDEX_OVERFLOW 4
+#define MOBA_STATUS_TIMEOUT 8     /* a bounded device wait gave up; outputs of that call are invalid */
 
 /* Bytes of device workspace moba_forward / moba_key_conv_centroid need for
  * `shape` (0 for an invalid shape).  The caller allocates it; its contents
