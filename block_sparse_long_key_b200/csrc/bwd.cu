@@ -18,7 +18,8 @@
 // S^T = K Q^T and dP^T = V dO^T, and feeds P^T and dS^T straight from the
 // accumulator registers into dV += P^T dO and dK += dS^T Q.  dS^T goes to
 // shared memory once for dQ = dS K, which every warp shares by 16x32 output
-// tiles and adds to the fp32 dQ buffer with vector reductions.
+// tiles and adds to the fp32 dQ buffer with 16-byte vector reductions (lane
+// pairs exchange halves so each lane holds 4 consecutive columns of a row).
 #include <algorithm>
 
 #include "common.cuh"
@@ -73,7 +74,6 @@ bwd_attn_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kg = warp % KG, rg = warp / KG;
   const size_t kv_stride = (size_t)h_kv * D;
-  const size_t q_stride = (size_t)h_q * D;
   const float scale = rsqrtf((float)D);
   const float scale_log2 = kLog2e * scale;
 
@@ -106,7 +106,7 @@ bwd_attn_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
       const int r = i / (D / 8), c = i % (D / 8);
       const int row = sm.row[buf][r];
       const bool ok = row >= 0;
-      const size_t off = ok ? (size_t)(row / h_q) * q_stride + (size_t)(row % h_q) * D + c * 8 : 0;
+      const size_t off = ok ? (size_t)row * D + c * 8 : 0;   // [T, H_q, D]: row t*H_q + h
       cp_async16_zfill(&sm.q[buf][r][c * 8], q + off, ok);
       cp_async16_zfill(&sm.dout[buf][r][c * 8], dout + off, ok);
     }
@@ -227,13 +227,25 @@ bwd_attn_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
           mma_bf16(acc[2 * nt2 + 1], a, b2, b3);
         }
       }
-      const int ra = m0 + (lane >> 2), rb = ra + 8;
-      const int rowa = sm.row[buf][ra], rowb = sm.row[buf][rb];
+      // Lane pairs swap halves so that each lane owns 4 consecutive columns
+      // of one row: one 16-byte reduction instead of two 8-byte ones.
+      const int q4 = lane & 3;
+      const bool even = (q4 & 1) == 0;
+      const int rr = m0 + (lane >> 2) + (even ? 0 : 8);
+      const int row = sm.row[buf][rr];
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt) {
-        const int col = c0 + nt * 8 + (lane & 3) * 2;
-        if (rowa >= 0) red_add_v2(dqacc + (size_t)rowa * D + col, acc[nt][0] * scale, acc[nt][1] * scale);
-        if (rowb >= 0) red_add_v2(dqacc + (size_t)rowb * D + col, acc[nt][2] * scale, acc[nt][3] * scale);
+        const float s0 = even ? acc[nt][2] : acc[nt][0];
+        const float s1 = even ? acc[nt][3] : acc[nt][1];
+        const float g0 = __shfl_xor_sync(0xffffffffu, s0, 1);
+        const float g1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+        const int col = c0 + nt * 8 + (even ? q4 : q4 - 1) * 2;
+        if (row >= 0) {
+          if (even)
+            red_add_v4(dqacc + (size_t)row * D + col, acc[nt][0] * scale, acc[nt][1] * scale, g0 * scale, g1 * scale);
+          else
+            red_add_v4(dqacc + (size_t)row * D + col, g0 * scale, g1 * scale, acc[nt][2] * scale, acc[nt][3] * scale);
+        }
       }
     }
     __syncthreads();

@@ -18,7 +18,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/moba.h"
+#include "moba.h"
 #include "launch.h"
 
 namespace {

@@ -32,9 +32,12 @@ cudaError_t launch_conv_centroid(const bf16* k, const float* conv_w, int conv_wi
                                  int h_kv, int d, int block_size, bf16* k_out, float* cent,
                                  bf16* cent_hi, bf16* cent_lo, cudaStream_t st);
 
+// Forward accumulator rows: O (d floats), l, 3 floats of padding.
+__host__ __device__ constexpr int oacc_stride(int d) { return d + 4; }
+
 cudaError_t launch_route(const bf16* q, const bf16* k, const bf16* cent_hi, const bf16* cent_lo,
                          const SeqPlan& p, int h_q, int h_kv, int d, int block_size, int topk,
-                         int32_t* sel_idx, float* mref, int32_t* flag, float* lacc, float* oacc,
+                         int32_t* sel_idx, float* mref, int32_t* flag, float* oacc,
                          int32_t* status, cudaStream_t st);
 
 cudaError_t launch_build_index(const int32_t* sel_idx, const SeqPlan& p, int h_q, int h_kv,
@@ -43,12 +46,10 @@ cudaError_t launch_build_index(const int32_t* sel_idx, const SeqPlan& p, int h_q
 
 cudaError_t launch_fwd_attn(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p,
                             const int32_t* ptr, const int32_t* rows, const float* mref, int h_q,
-                            int h_kv, int d, int block_size, float* oacc, float* lacc, int32_t* flag,
-                            cudaStream_t st);
+                            int h_kv, int d, int block_size, float* oacc, int32_t* flag, cudaStream_t st);
 
-cudaError_t launch_fwd_finalize(const float* oacc, const float* lacc, const float* mref,
-                                const int32_t* flag, int nrows, int d, bf16* out, float* lse,
-                                int32_t* flag_list, cudaStream_t st);
+cudaError_t launch_fwd_finalize(const float* oacc, const float* mref, const int32_t* flag, int nrows,
+                                int d, bf16* out, float* lse, int32_t* flag_list, cudaStream_t st);
 
 cudaError_t launch_fwd_fallback(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p,
                                 const int32_t* sel_idx, const int32_t* flag_list, int h_q, int h_kv,

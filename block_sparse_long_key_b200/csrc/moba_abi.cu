@@ -5,7 +5,7 @@
 #include <cstdint>
 #include <cstring>
 
-#include "../../include/moba.h"
+#include "moba.h"
 #include "common.cuh"
 #include "launch.h"
 
@@ -67,8 +67,7 @@ struct FwdBufs {
   bf16* lo;
   float* mref;
   int32_t* flag;
-  float* lacc;
-  float* oacc;
+  float* oacc;  // rows of oacc_stride(d) floats: O, l, padding
   int32_t* cnt;
   int32_t* ptr;
   int32_t* cursor;
@@ -87,8 +86,7 @@ FwdBufs carve_fwd(Carve& c, const moba_shape* s) {
   b.lo = c.take<bf16>(ncent);
   b.mref = c.take<float>(nrow);
   b.flag = c.take<int32_t>(nrow);
-  b.lacc = c.take<float>(nrow);
-  b.oacc = c.take<float>(nrow * s->head_dim);
+  b.oacc = c.take<float>(nrow * moba::oacc_stride(s->head_dim));
   b.cnt = c.take<int32_t>(nbk);
   b.ptr = c.take<int32_t>(nbk + 1);
   b.cursor = c.take<int32_t>(nbk);
@@ -241,7 +239,7 @@ int moba_forward(const void* q, const void* k, const void* v, const int32_t* cu_
                                       static_cast<bf16*>(k_conv_out), b.cent, b.hi, b.lo, st));
   STAGE_END(MOBA_STAGE_FWD_CENTROID);
   STAGE_BEGIN(MOBA_STAGE_FWD_ROUTE);
-  MOBA_TRY(moba::launch_route(kq, kk, b.hi, b.lo, plan, hq, hkv, d, B, topk, sel_idx, b.mref, b.flag, b.lacc, b.oacc,
+  MOBA_TRY(moba::launch_route(kq, kk, b.hi, b.lo, plan, hq, hkv, d, B, topk, sel_idx, b.mref, b.flag, b.oacc,
                               b.plan.status, st));
   STAGE_END(MOBA_STAGE_FWD_ROUTE);
   STAGE_BEGIN(MOBA_STAGE_FWD_INDEX);
@@ -249,11 +247,10 @@ int moba_forward(const void* q, const void* k, const void* v, const int32_t* cu_
                                     b.plan.status, st));
   STAGE_END(MOBA_STAGE_FWD_INDEX);
   STAGE_BEGIN(MOBA_STAGE_FWD_ATTN);
-  MOBA_TRY(moba::launch_fwd_attn(kq, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.lacc, b.flag,
-                                 st));
+  MOBA_TRY(moba::launch_fwd_attn(kq, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.flag, st));
   STAGE_END(MOBA_STAGE_FWD_ATTN);
   STAGE_BEGIN(MOBA_STAGE_FWD_FINALIZE);
-  MOBA_TRY(moba::launch_fwd_finalize(b.oacc, b.lacc, b.mref, b.flag, T * hq, d, static_cast<bf16*>(out), lse,
+  MOBA_TRY(moba::launch_fwd_finalize(b.oacc, b.mref, b.flag, T * hq, d, static_cast<bf16*>(out), lse,
                                      b.flag_list, st));
   MOBA_TRY(moba::launch_fwd_fallback(kq, kk, kv, plan, sel_idx, b.flag_list, hq, hkv, d, B, topk,
                                      static_cast<bf16*>(out), lse, st));
