@@ -175,10 +175,10 @@ KERNEL_SRC = {"fwd_attn": "fwd.cu", "bwd_attn": "bwd.cu", "fwd_route": "route.cu
               "fwd_finalize": "fwd.cu", "bwd_pre": "bwd.cu", "bwd_dq": "bwd.cu", "fwd_index": "index.cu",
               "bwd_index": "index.cu"}
 
-# Kernels of ours launched per step: forward 9 (plan, conv/centroid, route,
-# count, scan, fill, attention, finalize, fallback), backward 7 (plan, count,
-# scan, fill, preprocess, attention, dQ).
-LAUNCHES_PER_STEP = 16
+# Kernels of ours launched per step: forward 10 (plan, conv/centroid, route,
+# index count, prefix, scan, fill, attention, finalize, fallback), backward 4
+# (plan, preprocess, attention, dQ; the forward's block index is reused).
+LAUNCHES_PER_STEP = 14
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) timing
@@ -262,7 +262,8 @@ def run_ours(args):
     def step(qd, kd, vd, dod, cud, cw):
         _, _, _, k_used = moba.forward(qd, kd, vd, cud, B, topk, conv_w=cw, workspace=ws_f, out=out, lse=lse,
                                        sel_idx=sel, k_conv=kc)
-        moba.backward(qd, k_used, vd, out, lse, dod, sel, cud, B, workspace=ws_b, dq=dq, dk=dk, dv=dv)
+        moba.backward(qd, k_used, vd, out, lse, dod, sel, cud, B, workspace=ws_b, dq=dq, dk=dk, dv=dv,
+                      fwd_workspace=ws_f)
 
     for _ in range(args.warmup):
         step(g["q"], g["k"], g["v"], g["dout"], g["cu_seqlens"], conv_w)

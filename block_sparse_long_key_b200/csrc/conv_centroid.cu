@@ -8,12 +8,14 @@
 //    Formale": k'_t = k_t + SiLU(sum_{l=0}^{W-1} W_l (.) k_{t-l}), one filter
 //    per channel, causal (left zero padding at the sequence start).
 //
-// One CTA per (global block, KV head) reads the block's B key rows once with
-// 16-byte vector loads (D/8 threads per row), writes k' (bf16, round to
-// nearest even) when the conv is on, and the centroid of the (converted)
-// keys as fp32 plus a bf16 hi/lo split (hi = bf16(c), lo = bf16(c - hi))
-// that the tensor-core router uses to reach fp32-level score accuracy.
-// HBM-bound: algorithmic bytes per block = B*D*2 read (+ B*D*2 written).
+// Eight threads per (global block, KV head), each owning 8 channels: a
+// thread walks the block's rows in order with 16-byte loads (the 8 threads of
+// a block read one 128/256-byte row segment together), keeps the previous
+// W-1 rows of its channels in registers for the conv, writes k' and sums the
+// (converted) keys itself, so no shared memory and no barrier are needed.
+// The sum runs in ascending token order in fp32 and is divided by the block's
+// token count.  HBM-bound: algorithmic bytes per block = B*D*2 read
+// (+ B*D*2 written with conv) + centroid outputs.
 #include "common.cuh"
 #include "launch.h"
 
@@ -29,22 +31,18 @@ conv_centroid_kernel(const bf16* __restrict__ k, const float* __restrict__ conv_
                      const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch,
                      int nb_max, int h_kv, int block_size, bf16* __restrict__ k_out,
                      float* __restrict__ cent, bf16* __restrict__ cent_hi, bf16* __restrict__ cent_lo) {
-  constexpr int TPR = D / 8;            // threads per key row
-  constexpr int RPP = kThreads / TPR;   // rows per pass
-  __shared__ float s_part[RPP][D];
-
-  const int gb = blockIdx.x;
-  const int h = blockIdx.y;
-  if (gb >= __ldg(blk_off + batch)) return;
+  constexpr int TPB = D / 8;  // threads per block (8 channels each)
+  const long long gtid = (long long)blockIdx.x * kThreads + threadIdx.x;
+  const int c8 = (int)(gtid % TPB);
+  const long long bidx = gtid / TPB;
+  const int h = (int)(bidx / nb_max);
+  const int gb = (int)(bidx % nb_max);
+  if (h >= h_kv || gb >= __ldg(blk_off + batch)) return;
   const int s = upper_seq(blk_off, batch, gb);
   const int j = gb - __ldg(blk_off + s);
   const int seq0 = __ldg(cu + s);
   const int t0 = seq0 + j * block_size;
   const int t1 = min(t0 + block_size, __ldg(cu + s + 1));
-  const int nrows = t1 - t0;
-
-  const int c8 = threadIdx.x % TPR;
-  const int rr = threadIdx.x / TPR;
   const size_t row_stride = (size_t)h_kv * D;
   const bf16* kh = k + (size_t)h * D + c8 * 8;
 
@@ -53,10 +51,9 @@ conv_centroid_kernel(const bf16* __restrict__ k, const float* __restrict__ conv_
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 
   if (width == 0) {
-    for (int r = rr; r < nrows; r += RPP) {
-      uint4 u = __ldg(reinterpret_cast<const uint4*>(kh + (size_t)(t0 + r) * row_stride));
+    for (int t = t0; t < t1; ++t) {
       float f[8];
-      bf16x8_to_f32(u, f);
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kh + (size_t)t * row_stride)), f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] += f[i];
     }
@@ -67,54 +64,63 @@ conv_centroid_kernel(const bf16* __restrict__ k, const float* __restrict__ conv_
 #pragma unroll
       for (int i = 0; i < 8; ++i)
         w[l][i] = l < width ? __ldg(conv_w + ((size_t)h * D + c8 * 8 + i) * width + l) : 0.f;
-    bf16* ko = k_out + (size_t)h * D + c8 * 8;
-    for (int r = rr; r < nrows; r += RPP) {
-      const int t = t0 + r;
-      float x[8], kt[8];
+    // win[l] holds k_{t-1-l} (zero before the sequence start)
+    float win[kMaxWidth - 1][8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = 0.f;
+    for (int l = 0; l < kMaxWidth - 1; ++l) {
+      const int tp = t0 - 1 - l;
+      if (l + 1 < width && tp >= seq0) {
+        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kh + (size_t)tp * row_stride)), win[l]);
+      } else {
 #pragma unroll
-      for (int l = 0; l < kMaxWidth; ++l) {
-        if (l < width && t - l >= seq0) {
-          uint4 u = __ldg(reinterpret_cast<const uint4*>(kh + (size_t)(t - l) * row_stride));
-          float f[8];
-          bf16x8_to_f32(u, f);
-          if (l == 0) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) kt[i] = f[i];
-          }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) x[i] = fmaf(w[l][i], f[i], x[i]);
-        }
+        for (int i = 0; i < 8; ++i) win[l][i] = 0.f;
       }
+    }
+    bf16* ko = k_out + (size_t)h * D + c8 * 8;
+    for (int t = t0; t < t1; ++t) {
+      float cur[8], x[8];
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kh + (size_t)t * row_stride)), cur);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = w[0][i] * cur[i];
+#pragma unroll
+      for (int l = 1; l < kMaxWidth; ++l)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = fmaf(w[l][i], win[l - 1][i], x[i]);
       float y[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float silu = x[i] / (1.f + expf(-x[i]));
-        y[i] = kt[i] + silu;
-      }
-      uint4 packed = f32_to_bf16x8(y);
+      for (int i = 0; i < 8; ++i) y[i] = cur[i] + x[i] / (1.f + expf(-x[i]));
+      const uint4 packed = f32_to_bf16x8(y);
       *reinterpret_cast<uint4*>(ko + (size_t)t * row_stride) = packed;
       float yr[8];
       bf16x8_to_f32(packed, yr);  // the centroid averages the stored bf16 keys
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] += yr[i];
+#pragma unroll
+      for (int l = kMaxWidth - 2; l > 0; --l)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) win[l][i] = win[l - 1][i];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) win[0][i] = cur[i];
     }
   }
 
+  const float inv = 1.f / (float)(t1 - t0);
+  float c[8], lo[8];
+  bf16 hb[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) s_part[rr][c8 * 8 + i] = acc[i];
-  __syncthreads();
-  if (threadIdx.x < D) {
-    float sum = 0.f;
-    for (int g = 0; g < RPP; ++g) sum += s_part[g][threadIdx.x];
-    const float c = sum / (float)nrows;
-    const size_t o = ((size_t)h * nb_max + gb) * D + threadIdx.x;
-    cent[o] = c;
-    const bf16 hi = __float2bfloat16_rn(c);
-    cent_hi[o] = hi;
-    cent_lo[o] = __float2bfloat16_rn(c - __bfloat162float(hi));
+  for (int i = 0; i < 8; ++i) {
+    c[i] = acc[i] * inv;
+    hb[i] = __float2bfloat16_rn(c[i]);
+    lo[i] = c[i] - __bfloat162float(hb[i]);
   }
+  const size_t o = ((size_t)h * nb_max + gb) * D + c8 * 8;
+  reinterpret_cast<float4*>(cent + o)[0] = make_float4(c[0], c[1], c[2], c[3]);
+  reinterpret_cast<float4*>(cent + o)[1] = make_float4(c[4], c[5], c[6], c[7]);
+  float hf[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) hf[i] = __bfloat162float(hb[i]);
+  *reinterpret_cast<uint4*>(cent_hi + o) = f32_to_bf16x8(hf);
+  *reinterpret_cast<uint4*>(cent_lo + o) = f32_to_bf16x8(lo);
 }
 
 }  // namespace
@@ -123,15 +129,15 @@ cudaError_t launch_conv_centroid(const bf16* k, const float* conv_w, int conv_wi
                                  int h_kv, int d, int block_size, bf16* k_out, float* cent,
                                  bf16* cent_hi, bf16* cent_lo, cudaStream_t st) {
   if (conv_width > kMaxWidth) return cudaErrorInvalidValue;
-  dim3 grid(p.nb_max, h_kv);
+  const long long threads = (long long)p.nb_max * h_kv * (d / 8);
+  const int grid = (int)((threads + kThreads - 1) / kThreads);
+  if (grid == 0) return cudaSuccess;
   if (d == 64)
-    conv_centroid_kernel<64><<<grid, kThreads, 0, st>>>(k, conv_w, conv_width, p.cu, p.blk_off, p.batch,
-                                                        p.nb_max, h_kv, block_size, k_out, cent,
-                                                        cent_hi, cent_lo);
+    conv_centroid_kernel<64><<<grid, kThreads, 0, st>>>(k, conv_w, conv_width, p.cu, p.blk_off, p.batch, p.nb_max,
+                                                        h_kv, block_size, k_out, cent, cent_hi, cent_lo);
   else
-    conv_centroid_kernel<128><<<grid, kThreads, 0, st>>>(k, conv_w, conv_width, p.cu, p.blk_off, p.batch,
-                                                         p.nb_max, h_kv, block_size, k_out, cent,
-                                                         cent_hi, cent_lo);
+    conv_centroid_kernel<128><<<grid, kThreads, 0, st>>>(k, conv_w, conv_width, p.cu, p.blk_off, p.batch, p.nb_max,
+                                                         h_kv, block_size, k_out, cent, cent_hi, cent_lo);
   return cudaGetLastError();
 }
 

@@ -12,10 +12,17 @@
 // query, its output and its statistics directly.  Own-block picks are
 // included; the attention kernels apply the causal cut for them.
 //
-// Three passes: count (one atomic per pick), exclusive scan of the counts
-// (one CTA), fill (one atomic per pick to claim a slot).  The order of rows
-// inside a bucket is therefore not deterministic; no result depends on it
-// beyond fp32 summation order.  Integer work, bound by the atomics.
+// Main path (a KV head's blocks fit a shared-memory histogram): the picks of
+// one KV head are cut into chunks of kChunkTokens tokens; one CTA per
+// (chunk, KV head) counts its picks per block with shared-memory atomics and
+// writes that histogram row; a per-bucket pass turns the rows into each
+// chunk's starting offset inside the bucket; a one-CTA scan gives the bucket
+// starts; the fill pass re-reads the picks and places them with
+// shared-memory cursors.  Global traffic: the picks twice, the rows once, the
+// histogram rows a few times.  Fallback (huge block counts, or no chunk
+// buffer): one global atomic per pick to count and one to claim a slot.  The
+// order of rows inside a bucket is not deterministic; no result depends on
+// it beyond fp32 summation order.
 #include <algorithm>
 
 #include "common.cuh"
@@ -26,6 +33,9 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kScanThreads = 1024;
+constexpr int kChunkTokens = 1024;
+constexpr int kBatch = 8;  // picks per thread with their loads in flight together
+constexpr int kMaxSmemBuckets = 16384;  // 64 KB of shared-memory counters
 
 // Returns the bucket of pick `e` (row * topk + slot) or -1 if the slot is
 // empty or invalid (invalid entries raise kStatusBadSelIdx).
@@ -103,16 +113,157 @@ fill_kernel(const int32_t* __restrict__ sel_idx, long long npicks, int topk, int
   }
 }
 
+// ---- shared-memory privatised path
+
+// Pick i of chunk (tokens [ta, ta + kChunkTokens)) of KV head kvh: its
+// position in sel_idx, or -1 past the chunk / outside every sequence.
+// Also returns the pick's token and query row id.
+__device__ __forceinline__ long long chunk_pick_pos(int i, int n, int ta, int kvh, int group, int topk, int h_q,
+                                                    int seq_end, int& t, int& row) {
+  if (i >= n) return -1;
+  const int per_tok = group * topk;
+  t = ta + i / per_tok;
+  if (t >= seq_end) return -1;
+  const int rem = i - (t - ta) * per_tok;
+  row = t * h_q + kvh * group + rem / topk;
+  return (long long)row * topk + rem % topk;
+}
+
+// Local bucket (blk_off[s] + j) of the pick at `e` holding block j, or -1 if
+// the slot is empty or invalid (invalid entries raise kStatusBadSelIdx).
+__device__ __forceinline__ int chunk_pick_bucket(long long e, int t, int j, int block_size, const int32_t* cu,
+                                                 const int32_t* blk_off, int batch, int32_t* status) {
+  if (e < 0) return -1;
+  if (j < 0) {
+    if (j != -1) set_status(status, kStatusBadSelIdx);
+    return -1;
+  }
+  const int s = upper_seq(cu, batch, t);
+  if (j > (t - __ldg(cu + s)) / block_size) {
+    set_status(status, kStatusBadSelIdx);
+    return -1;
+  }
+  return __ldg(blk_off + s) + j;
+}
+
+__global__ void __launch_bounds__(kThreads)
+chunk_count_kernel(const int32_t* __restrict__ sel_idx, int total_tokens, int topk, int h_q, int group,
+                   int block_size, const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch,
+                   int nb_max, int nchunks, int32_t* __restrict__ chunk_cnt, int32_t* __restrict__ status) {
+  extern __shared__ int32_t hist[];
+  const int c = blockIdx.x, kvh = blockIdx.y;
+  for (int b = threadIdx.x; b < nb_max; b += kThreads) hist[b] = 0;
+  __syncthreads();
+  const int ta = c * kChunkTokens;
+  const int n = max(0, min(kChunkTokens, total_tokens - ta)) * group * topk;
+  const int seq_end = __ldg(cu + batch);
+  for (int i0 = threadIdx.x; i0 < n; i0 += kThreads * kBatch) {
+    long long e[kBatch];
+    int j[kBatch], t[kBatch], row[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      e[u] = chunk_pick_pos(i0 + u * kThreads, n, ta, kvh, group, topk, h_q, seq_end, t[u], row[u]);
+      j[u] = e[u] >= 0 ? __ldg(sel_idx + e[u]) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int lb = chunk_pick_bucket(e[u], t[u], j[u], block_size, cu, blk_off, batch, status);
+      if (lb >= 0) atomicAdd(hist + lb, 1);
+    }
+  }
+  __syncthreads();
+  int32_t* dst = chunk_cnt + ((size_t)kvh * nchunks + c) * nb_max;
+  for (int b = threadIdx.x; b < nb_max; b += kThreads) dst[b] = hist[b];
+}
+
+// Per bucket: chunk counts -> exclusive prefix over chunks (in place), total
+// into cnt.
+__global__ void __launch_bounds__(kThreads)
+chunk_prefix_kernel(int32_t* __restrict__ chunk_cnt, int nb_max, int nchunks, int h_kv, int32_t* __restrict__ cnt) {
+  const int b = blockIdx.x * kThreads + threadIdx.x;
+  if (b >= h_kv * nb_max) return;
+  const int kvh = b / nb_max, lb = b % nb_max;
+  int32_t* col = chunk_cnt + (size_t)kvh * nchunks * nb_max + lb;
+  int run = 0;
+  for (int c = 0; c < nchunks; ++c) {
+    const int v = col[(size_t)c * nb_max];
+    col[(size_t)c * nb_max] = run;
+    run += v;
+  }
+  cnt[b] = run;
+}
+
+__global__ void __launch_bounds__(kThreads)
+chunk_fill_kernel(const int32_t* __restrict__ sel_idx, int total_tokens, int topk, int h_q, int group,
+                  int block_size, const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch,
+                  int nb_max, int nchunks, const int32_t* __restrict__ chunk_cnt, const int32_t* __restrict__ ptr,
+                  int32_t* __restrict__ rows, int32_t* __restrict__ status) {
+  extern __shared__ int32_t cursor[];
+  const int c = blockIdx.x, kvh = blockIdx.y;
+  const int32_t* src = chunk_cnt + ((size_t)kvh * nchunks + c) * nb_max;
+  const int32_t* base = ptr + (size_t)kvh * nb_max;
+  for (int b = threadIdx.x; b < nb_max; b += kThreads) cursor[b] = __ldg(base + b) + __ldg(src + b);
+  __syncthreads();
+  const int ta = c * kChunkTokens;
+  const int n = max(0, min(kChunkTokens, total_tokens - ta)) * group * topk;
+  const int seq_end = __ldg(cu + batch);
+  for (int i0 = threadIdx.x; i0 < n; i0 += kThreads * kBatch) {
+    long long e[kBatch];
+    int j[kBatch], t[kBatch], row[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      e[u] = chunk_pick_pos(i0 + u * kThreads, n, ta, kvh, group, topk, h_q, seq_end, t[u], row[u]);
+      j[u] = e[u] >= 0 ? __ldg(sel_idx + e[u]) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      // invalid entries were reported by the count pass
+      const int lb = chunk_pick_bucket(e[u], t[u], j[u], block_size, cu, blk_off, batch, status);
+      if (lb >= 0) rows[atomicAdd(cursor + lb, 1)] = row[u];
+    }
+  }
+}
+
 }  // namespace
+
+size_t index_chunk_ints(int total_tokens, int h_kv, int nb_max) {
+  if (nb_max > kMaxSmemBuckets) return 0;
+  const size_t nchunks = ((size_t)total_tokens + kChunkTokens - 1) / kChunkTokens;
+  return (size_t)h_kv * nchunks * nb_max;
+}
 
 cudaError_t launch_build_index(const int32_t* sel_idx, const SeqPlan& p, int h_q, int h_kv, int block_size,
                                int topk, int32_t* cnt, int32_t* ptr, int32_t* cursor, int32_t* rows,
-                               int32_t* status, cudaStream_t st) {
+                               int32_t* status, cudaStream_t st, int32_t* chunk_cnt) {
   const int nbk = h_kv * p.nb_max;
   const long long npicks = (long long)p.total_tokens * h_q * topk;
-  cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(int32_t) * (size_t)nbk, st);
-  if (e != cudaSuccess) return e;
   const int group = h_q / h_kv;
+  cudaError_t e;
+  if (chunk_cnt != nullptr && p.nb_max <= kMaxSmemBuckets && p.total_tokens > 0) {
+    const int nchunks = (p.total_tokens + kChunkTokens - 1) / kChunkTokens;
+    const size_t smem = sizeof(int32_t) * (size_t)p.nb_max;
+    if ((e = cudaFuncSetAttribute(chunk_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+        cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(chunk_fill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+        cudaSuccess)
+      return e;
+    dim3 grid(nchunks, h_kv);
+    chunk_count_kernel<<<grid, kThreads, smem, st>>>(sel_idx, p.total_tokens, topk, h_q, group, block_size, p.cu,
+                                                     p.blk_off, p.batch, p.nb_max, nchunks, chunk_cnt, status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    chunk_prefix_kernel<<<(nbk + kThreads - 1) / kThreads, kThreads, 0, st>>>(chunk_cnt, p.nb_max, nchunks, h_kv,
+                                                                              cnt);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    scan_kernel<<<1, kScanThreads, 0, st>>>(cnt, nbk, ptr, cursor);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    chunk_fill_kernel<<<grid, kThreads, smem, st>>>(sel_idx, p.total_tokens, topk, h_q, group, block_size, p.cu,
+                                                    p.blk_off, p.batch, p.nb_max, nchunks, chunk_cnt, ptr, rows,
+                                                    status);
+    return cudaGetLastError();
+  }
+  e = cudaMemsetAsync(cnt, 0, sizeof(int32_t) * (size_t)nbk, st);
+  if (e != cudaSuccess) return e;
   const int grid = (int)std::min<long long>((npicks + kThreads - 1) / kThreads, 148LL * 16);
   if (npicks > 0) {
     count_kernel<<<grid, kThreads, 0, st>>>(sel_idx, npicks, topk, h_q, group, block_size, p.cu, p.blk_off,

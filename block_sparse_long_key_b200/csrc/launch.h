@@ -40,9 +40,13 @@ cudaError_t launch_route(const bf16* q, const bf16* k, const bf16* cent_hi, cons
                          int32_t* sel_idx, float* mref, int32_t* flag, float* oacc,
                          int32_t* status, cudaStream_t st);
 
+// chunk_cnt (optional, index_chunk_ints() int32) selects the shared-memory
+// privatised path; nullptr, or a zero size from index_chunk_ints(), uses one
+// global atomic per pick.
+size_t index_chunk_ints(int total_tokens, int h_kv, int nb_max);
 cudaError_t launch_build_index(const int32_t* sel_idx, const SeqPlan& p, int h_q, int h_kv,
                                int block_size, int topk, int32_t* cnt, int32_t* ptr, int32_t* cursor,
-                               int32_t* rows, int32_t* status, cudaStream_t st);
+                               int32_t* rows, int32_t* status, cudaStream_t st, int32_t* chunk_cnt = nullptr);
 
 cudaError_t launch_fwd_attn(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p,
                             const int32_t* ptr, const int32_t* rows, const float* mref, int h_q,

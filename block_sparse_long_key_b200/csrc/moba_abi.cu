@@ -72,6 +72,7 @@ struct FwdBufs {
   int32_t* ptr;
   int32_t* cursor;
   int32_t* rows;
+  int32_t* chunk_cnt;  // per-chunk bucket histograms of the index builder (may be null)
   int32_t* flag_list;
 };
 
@@ -91,6 +92,8 @@ FwdBufs carve_fwd(Carve& c, const moba_shape* s) {
   b.ptr = c.take<int32_t>(nbk + 1);
   b.cursor = c.take<int32_t>(nbk);
   b.rows = c.take<int32_t>(nrow * s->topk);
+  const size_t nch = moba::index_chunk_ints(s->total_tokens, s->h_kv, nb_max_of(s));
+  b.chunk_cnt = nch ? c.take<int32_t>(nch) : nullptr;
   b.flag_list = c.take<int32_t>(nrow + 1);
   return b;
 }
@@ -101,6 +104,7 @@ struct BwdBufs {
   int32_t* ptr;
   int32_t* cursor;
   int32_t* rows;
+  int32_t* chunk_cnt;
   float* dsum;
   float* dqacc;
 };
@@ -114,6 +118,8 @@ BwdBufs carve_bwd(Carve& c, const moba_shape* s) {
   b.ptr = c.take<int32_t>(nbk + 1);
   b.cursor = c.take<int32_t>(nbk);
   b.rows = c.take<int32_t>(nrow * s->topk);
+  const size_t nch = moba::index_chunk_ints(s->total_tokens, s->h_kv, nb_max_of(s));
+  b.chunk_cnt = nch ? c.take<int32_t>(nch) : nullptr;
   b.dsum = c.take<float>(nrow);
   b.dqacc = c.take<float>(nrow * s->head_dim);
   return b;
@@ -244,7 +250,7 @@ int moba_forward(const void* q, const void* k, const void* v, const int32_t* cu_
   STAGE_END(MOBA_STAGE_FWD_ROUTE);
   STAGE_BEGIN(MOBA_STAGE_FWD_INDEX);
   MOBA_TRY(moba::launch_build_index(sel_idx, plan, hq, hkv, B, topk, b.cnt, b.ptr, b.cursor, b.rows,
-                                    b.plan.status, st));
+                                    b.plan.status, st, b.chunk_cnt));
   STAGE_END(MOBA_STAGE_FWD_INDEX);
   STAGE_BEGIN(MOBA_STAGE_FWD_ATTN);
   MOBA_TRY(moba::launch_fwd_attn(kq, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.flag, st));
@@ -272,18 +278,19 @@ int moba_build_index(const int32_t* sel_idx, const int32_t* cu_seqlens, const mo
   moba::SeqPlan plan;
   if ((rc = begin_plan(b.plan, cu_seqlens, shape, st, &plan, -1)) != MOBA_OK) return rc;
   MOBA_TRY(moba::launch_build_index(sel_idx, plan, shape->h_q, shape->h_kv, shape->block_size, shape->topk, b.cnt,
-                                    blk_ptr, b.cursor, blk_rows, b.plan.status, st));
+                                    blk_ptr, b.cursor, blk_rows, b.plan.status, st, b.chunk_cnt));
   return MOBA_OK;
 }
 
 int moba_backward(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
                   const int32_t* sel_idx, const int32_t* cu_seqlens, const moba_shape* shape, void* dq, void* dk,
-                  void* dv, void* workspace, size_t workspace_bytes, void* stream) {
+                  void* dv, void* workspace, size_t workspace_bytes, const void* fwd_workspace, void* stream) {
   if (!shape_ok(shape)) return MOBA_EINVAL;
   if (shape->total_tokens == 0) return MOBA_OK;
   int rc;
   if ((rc = check_ptrs({q, k, v, out, lse, dout, sel_idx, cu_seqlens, dq, dk, dv})) != MOBA_OK) return rc;
   if ((rc = check_ws(workspace, workspace_bytes, moba_bwd_workspace_size(shape))) != MOBA_OK) return rc;
+  if (fwd_workspace && !aligned(fwd_workspace, kAlign)) return MOBA_EALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Carve c;
   c.base = static_cast<char*>(workspace);
@@ -291,9 +298,20 @@ int moba_backward(const void* q, const void* k, const void* v, const void* out, 
   moba::SeqPlan plan;
   if ((rc = begin_plan(b.plan, cu_seqlens, shape, st, &plan, MOBA_STAGE_BWD_PLAN)) != MOBA_OK) return rc;
   const int T = shape->total_tokens, hq = shape->h_q, hkv = shape->h_kv, d = shape->head_dim;
+  const int32_t* ptr = b.ptr;
+  const int32_t* rows = b.rows;
   STAGE_BEGIN(MOBA_STAGE_BWD_INDEX);
-  MOBA_TRY(moba::launch_build_index(sel_idx, plan, hq, hkv, shape->block_size, shape->topk, b.cnt, b.ptr, b.cursor,
-                                    b.rows, b.plan.status, st));
+  if (fwd_workspace) {
+    // Reuse the block index the forward built in its workspace.
+    Carve cf;
+    cf.base = static_cast<char*>(const_cast<void*>(fwd_workspace));
+    FwdBufs f = carve_fwd(cf, shape);
+    ptr = f.ptr;
+    rows = f.rows;
+  } else {
+    MOBA_TRY(moba::launch_build_index(sel_idx, plan, hq, hkv, shape->block_size, shape->topk, b.cnt, b.ptr, b.cursor,
+                                      b.rows, b.plan.status, st, b.chunk_cnt));
+  }
   STAGE_END(MOBA_STAGE_BWD_INDEX);
   STAGE_BEGIN(MOBA_STAGE_BWD_PRE);
   MOBA_TRY(moba::launch_bwd_pre(static_cast<const bf16*>(out), static_cast<const bf16*>(dout), T * hq, d, b.dsum,
@@ -301,8 +319,8 @@ int moba_backward(const void* q, const void* k, const void* v, const void* out, 
   STAGE_END(MOBA_STAGE_BWD_PRE);
   STAGE_BEGIN(MOBA_STAGE_BWD_ATTN);
   MOBA_TRY(moba::launch_bwd_attn(static_cast<const bf16*>(q), static_cast<const bf16*>(k),
-                                 static_cast<const bf16*>(v), static_cast<const bf16*>(dout), lse, b.dsum, plan, b.ptr,
-                                 b.rows, hq, hkv, d, shape->block_size, b.dqacc, static_cast<bf16*>(dk),
+                                 static_cast<const bf16*>(v), static_cast<const bf16*>(dout), lse, b.dsum, plan, ptr,
+                                 rows, hq, hkv, d, shape->block_size, b.dqacc, static_cast<bf16*>(dk),
                                  static_cast<bf16*>(dv), st));
   STAGE_END(MOBA_STAGE_BWD_ATTN);
   STAGE_BEGIN(MOBA_STAGE_BWD_DQ);

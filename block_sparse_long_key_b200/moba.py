@@ -62,7 +62,7 @@ def lib() -> ctypes.CDLL:
         L.moba_forward.restype = I
         L.moba_build_index.argtypes = [P, P, F, P, P, P, S, P]
         L.moba_build_index.restype = I
-        L.moba_backward.argtypes = [P, P, P, P, P, P, P, P, F, P, P, P, P, S, P]
+        L.moba_backward.argtypes = [P, P, P, P, P, P, P, P, F, P, P, P, P, S, P, P]
         L.moba_backward.restype = I
         L.moba_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), I]
         L.moba_set_stage_events.restype = I
@@ -198,8 +198,11 @@ def build_index(sel_idx, cu_seqlens, h_kv: int, block_size: int, workspace=None)
 
 
 def backward(q, k, v, out, lse, dout, sel_idx, cu_seqlens, block_size: int, workspace=None,
-             dq=None, dk=None, dv=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """MoBA backward with the selection fixed.  Returns (dq, dk, dv)."""
+             dq=None, dk=None, dv=None, fwd_workspace=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """MoBA backward with the selection fixed.  Returns (dq, dk, dv).
+
+    ``fwd_workspace``: the workspace of the forward call that produced
+    ``sel_idx`` (untouched since); its block index is reused."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _need(t, torch.bfloat16, n, 3)
     _need(lse, torch.float32, "lse", 2)
@@ -213,7 +216,7 @@ def backward(q, k, v, out, lse, dout, sel_idx, cu_seqlens, block_size: int, work
     ws = workspace if workspace is not None else alloc_workspace(bwd_workspace_size(shape), q.device)
     rc = lib().moba_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(sel_idx),
                              _ptr(cu_seqlens), ctypes.byref(shape), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
-                             _stream())
+                             _ptr(fwd_workspace), _stream())
     _check(rc, "moba_backward")
     return dq, dk, dv
 

@@ -195,10 +195,15 @@ int moba_build_index_noalloc(const int32_t* sel_idx, const int32_t* cu_seqlens, 
  *                    of each group).  The gradient stops at k': the key
  *                    convolution's own backward is not part of this call.
  *  workspace         >= moba_bwd_workspace_size(shape) bytes
+ *  fwd_workspace     optional (NULL: rebuild the block index from sel_idx).
+ *                    The workspace of the moba_forward call that produced
+ *                    sel_idx, same shape, untouched since: its block index
+ *                    is reused instead of being rebuilt.  Read only.
  */
 int moba_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
                   const void* dout, const int32_t* sel_idx, const int32_t* cu_seqlens, const moba_shape* shape,
-                  void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, void* stream);
+                  void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                  const void* fwd_workspace, void* stream);
 
 /*
  * Optional stage timing for benchmarks.  While a table is installed on the

@@ -78,8 +78,9 @@ def test_argument_errors_return_codes_without_a_device(L):
     # the conv output may not alias the keys
     assert f(ok, ok, ok, ok, ctypes.byref(s), ok, 4, ok, ok, ok, ok, ok, big, None) == moba.MOBA_EINVAL
     b = L.moba_backward
-    assert b(ok, ok, ok, ok, ok, ok, ok, ok, ctypes.byref(s), ok, None, ok, ok, big, None) == moba.MOBA_EINVAL
-    assert b(ok, ok, ok, ok, ok, ok, ok, ok, ctypes.byref(s), ok, ok, ok, ok, 16, None) == moba.MOBA_EWORKSPACE
+    assert b(ok, ok, ok, ok, ok, ok, ok, ok, ctypes.byref(s), ok, None, ok, ok, big, None, None) == moba.MOBA_EINVAL
+    assert b(ok, ok, ok, ok, ok, ok, ok, ok, ctypes.byref(s), ok, ok, ok, ok, 16, None, None) == moba.MOBA_EWORKSPACE
+    assert b(ok, ok, ok, ok, ok, ok, ok, ok, ctypes.byref(s), ok, ok, ok, ok, big, mis, None) == moba.MOBA_EALIGN
     assert L.moba_build_index(ok, ok, ctypes.byref(s), ok, None, ok, big, None) == moba.MOBA_EINVAL
     assert L.moba_key_conv_centroid(ok, None, 0, ok, ctypes.byref(s), None, None, ok, big, None) == moba.MOBA_EINVAL
     st = ctypes.c_int32(0)

@@ -233,3 +233,25 @@ def test_full_size_sampled_rows(dev, name):
         s_r = pu.row_dq_error_scale(ref["q"], ref["k"], ref["v"], do32, sel_use, ref["cu"], w.block_size, rows,
                                     o_ref[idx], lse_ref[idx])
         pu.check_grad(pu.to64(dq)[idx], dq_r, s_r, "dq " + name)
+
+
+@pytest.mark.parametrize("case", [SMALL[1], SMALL[3]], ids=_ids)
+def test_backward_reusing_forward_index_matches_oracle(dev, case):
+    w, x = _inputs(case)
+    g = _gpu(x, dev)
+    shape = moba.shape_of(g["q"], g["k"], g["cu_seqlens"], w.block_size, w.topk)
+    wsf = moba.alloc_workspace(moba.fwd_workspace_size(shape), dev)
+    out, lse, sel, k_used = moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], w.block_size, w.topk,
+                                         conv_w=g.get("conv_w"), workspace=wsf)
+    dq, dk, dv = moba.backward(g["q"], k_used, g["v"], out, lse, g["dout"], sel, g["cu_seqlens"], w.block_size,
+                               fwd_workspace=wsf)
+    torch.cuda.synchronize()
+    ref = pu.oracle_forward(x, w.block_size, w.topk)
+    assert not pu.selection_mismatch_rows(sel.cpu().numpy(), ref["sel"], ref["gap"])
+    do64 = x["dout"].double().numpy()
+    dq_r, dk_r, dv_r = orc.attention_backward(ref["q"], ref["k"], ref["v"], do64, ref["sel"], ref["cu"], w.block_size)
+    sq, sk, sv = pu.grad_error_scales(ref["q"], ref["k"], ref["v"], do64, ref["sel"], ref["cu"], w.block_size,
+                                      ref["lse"], ref["o"])
+    pu.check_grad(pu.to64(dq), dq_r, sq, "dq reuse")
+    pu.check_grad(pu.to64(dk), dk_r, sk, "dk reuse")
+    pu.check_grad(pu.to64(dv), dv_r, sv, "dv reuse")
