@@ -22,13 +22,12 @@
 // t: tcgen05.ld hands it that row's NC scores in registers.  Scores above the
 // thread's running threshold (the worst of its current k-1 best) go to a
 // small per-thread candidate buffer in shared memory; the whole warp flushes
-// the buffers together.  The k-1 kept entries sit unsorted in shared memory
-// ([slot][thread], so every access is bank-conflict free) in groups of 8
-// whose worst entries are tracked in registers: admitting a candidate
-// overwrites the worst slot and rescans one group plus the group minima, a
-// fixed 8 + k/8 steps whatever the data (a sorted list would shift up to k-1
-// entries, and a warp pays for its slowest lane).  Order: higher score first,
-// equal scores by lower block index.
+// the buffers together.  The k-1 kept entries form a binary min-heap of
+// 64-bit keys (order-preserving score bits << 32 | ~block index, so a larger
+// key is a better block: higher score, then lower index) in shared memory
+// ([slot][thread], bank-conflict free); admitting a candidate replaces the
+// root and sifts it down a fixed log2(k) levels whatever the data (a sorted
+// list would shift up to k-1 entries, and a warp pays for its slowest lane).
 //
 // Side outputs for the forward: mref = a lower bound of the query's largest
 // attention logit, max(best kept score, q_i.k_i) / sqrt(d) (a block mean never
@@ -43,7 +42,10 @@ namespace {
 
 constexpr int kTM = kRouteTile;  // query rows per CTA (= TMEM lanes)
 constexpr int kThreads = 128;
-constexpr int kGroup = 8;        // kept-list slots per group
+constexpr uint64_t kKeyMax = ~0ull;  // heap padding: never the minimum
+// An empty live slot: the key of score -inf (below every finite score), so
+// the root's score reads back as -inf until k-1 blocks have been admitted.
+constexpr uint64_t kKeyEmpty = (uint64_t)0x007fffffu << 32;
 constexpr uint32_t kFull = 0xffffffffu;
 
 template <int D, int NC, int LISTN>
@@ -56,12 +58,11 @@ struct RouteLayout {
   static constexpr uint32_t C_REGION = NC * 128;
   static constexpr uint32_t C_MAT = KB * C_REGION;       // hi or lo of one chunk
   static constexpr uint32_t C_BUF = 2 * C_MAT;           // hi + lo
-  static constexpr uint32_t LV_OFF = C_OFF + 2 * C_BUF;
-  static constexpr uint32_t LI_OFF = LV_OFF + LISTN * kThreads * 4;
-  static constexpr uint32_t BV_OFF = LI_OFF + LISTN * kThreads * 4;
+  static constexpr uint32_t HP_OFF = C_OFF + 2 * C_BUF;           // heap keys [LISTN][kThreads] u64
+  static constexpr uint32_t BV_OFF = HP_OFF + LISTN * kThreads * 8;
   static constexpr uint32_t BI_OFF = BV_OFF + kBuf * kThreads * 4;
   static constexpr uint32_t MB_OFF = BI_OFF + kBuf * kThreads * 4;
-  static_assert(LISTN % kGroup == 0, "kept list is whole groups");
+  static_assert((LISTN & (LISTN - 1)) == 0, "heap is a complete tree of LISTN - 1 nodes");
   static constexpr uint32_t HOLD_OFF = MB_OFF + 16;
   static constexpr uint32_t FLAG_OFF = HOLD_OFF + 4;
   static constexpr uint32_t BYTES = FLAG_OFF + 12;
@@ -69,6 +70,14 @@ struct RouteLayout {
   static_assert(C_REGION % 1024 == 0 && Q_REGION % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
   static_assert(TMEM_COLS >= 32 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation is a power of two");
 };
+
+__device__ __forceinline__ uint32_t order_bits(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float from_order_bits(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
 
 template <int D, int NC, int LISTN>
 __global__ void __launch_bounds__(kThreads)
@@ -79,11 +88,13 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
              float* __restrict__ mref, int32_t* __restrict__ flag, float* __restrict__ oacc,
              int32_t* __restrict__ status) {
   using Ly = RouteLayout<D, NC, LISTN>;
+  // Sift depth of a complete tree with LISTN - 1 nodes (children of the
+  // deepest internal node still lie below LISTN - 1).
+  constexpr int kHeapDepth = LISTN == 64 ? 5 : (LISTN == 32 ? 4 : (LISTN == 16 ? 3 : 2));
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(sm);
-  float* lv = reinterpret_cast<float*>(sm + Ly::LV_OFF);
-  int32_t* li = reinterpret_cast<int32_t*>(sm + Ly::LI_OFF);
+  uint64_t* heap = reinterpret_cast<uint64_t*>(sm + Ly::HP_OFF);
   float* bv = reinterpret_cast<float*>(sm + Ly::BV_OFF);
   int32_t* bi = reinterpret_cast<int32_t*>(sm + Ly::BI_OFF);
   const uint32_t mbar0 = sbase + Ly::MB_OFF;
@@ -135,46 +146,10 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   // ---- per-thread selection state; TMEM + barriers
   const bool row_ok = tid < nrows;
   const int my_b = row_ok ? (p0 + tid) / block_size : 0;
-  // Kept list: k1 live slots start as (-inf, INT_MAX) placeholders, the padding
-  // slots up to LISTN hold +inf and are never evicted.
-  constexpr int NG = LISTN / kGroup;
-  float gv[NG];
-  int gj[NG], gs[NG];
-#pragma unroll
-  for (int g = 0; g < NG; ++g) {
-    gv[g] = INFINITY;
-    gj[g] = -1;
-    gs[g] = g * kGroup;
-#pragma unroll
-    for (int e = 0; e < kGroup; ++e) {
-      const int sl = g * kGroup + e;
-      const bool live = sl < k1;
-      lv[sl * kThreads + tid] = live ? -INFINITY : INFINITY;
-      li[sl * kThreads + tid] = live ? 0x7fffffff : -1;
-      if (live && gv[g] == INFINITY) {
-        gv[g] = -INFINITY;
-        gj[g] = 0x7fffffff;
-        gs[g] = sl;
-      }
-    }
-  }
-  // worst kept entry (the threshold) = worst of the group minima
-  float tau = -INFINITY;
-  int tau_j = 0x7fffffff, tau_s = 0;
-  auto worse = [](float av, int aj, float bv, int bj) { return av < bv || (av == bv && aj > bj); };
-  auto refresh_tau = [&]() {
-    tau = gv[0];
-    tau_j = gj[0];
-    tau_s = gs[0];
-#pragma unroll
-    for (int g = 1; g < NG; ++g)
-      if (worse(gv[g], gj[g], tau, tau_j)) {
-        tau = gv[g];
-        tau_j = gj[g];
-        tau_s = gs[g];
-      }
-  };
-  refresh_tau();
+  // Min-heap of the kept keys: k1 live slots start empty (score -inf),
+  // padding slots up to LISTN-1 hold kKeyMax and never surface.
+  for (int sl = 0; sl < LISTN; ++sl) heap[sl * kThreads + tid] = sl < k1 ? kKeyEmpty : kKeyMax;
+  float tau = -INFINITY;  // score of the root (the worst kept entry)
   int cnt = 0;
   if (tid == 0) {
     tc::mbar_init(mbar0, 1);
@@ -196,35 +171,29 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
   constexpr uint32_t idesc = tc::idesc_bf16_f32(kTM, NC);
 
-  // Admit (x, j), x > tau: overwrite the worst slot, rescan its group, then
-  // the group minima.  Candidates arrive in ascending j, so a score equal to
-  // the threshold never displaces it (lower index wins ties).
+  // Admit (x, j), x > tau: replace the root and sift it down.  Candidates
+  // arrive in ascending j, so a score equal to the threshold never displaces
+  // it (lower index wins ties): the strict test on the score is exact.
   auto admit = [&](float x, int j) {
-    const int s0 = tau_s;
-    lv[s0 * kThreads + tid] = x;
-    li[s0 * kThreads + tid] = j;
-    const int g0 = s0 / kGroup;
-    float mv = INFINITY;
-    int mj = -1, ms = g0 * kGroup;
+    const uint64_t key = ((uint64_t)order_bits(x) << 32) | (uint64_t)(0xffffffffu - (uint32_t)j);
+    int pos = 0;
+    bool done = false;
 #pragma unroll
-    for (int e = 0; e < kGroup; ++e) {
-      const int sl = g0 * kGroup + e;
-      const float v = lv[sl * kThreads + tid];
-      const int jj = li[sl * kThreads + tid];
-      if (worse(v, jj, mv, mj)) {
-        mv = v;
-        mj = jj;
-        ms = sl;
+    for (int lvl = 0; lvl < kHeapDepth; ++lvl) {
+      const int c1 = 2 * pos + 1;
+      const uint64_t k1v = heap[c1 * kThreads + tid];
+      const uint64_t k2v = heap[(c1 + 1) * kThreads + tid];
+      const bool left = k1v < k2v;
+      const uint64_t km = left ? k1v : k2v;
+      if (!done && km < key) {
+        heap[pos * kThreads + tid] = km;
+        pos = left ? c1 : c1 + 1;
+      } else {
+        done = true;
       }
     }
-#pragma unroll
-    for (int g = 0; g < NG; ++g)
-      if (g == g0) {
-        gv[g] = mv;
-        gj[g] = mj;
-        gs[g] = ms;
-      }
-    refresh_tau();
+    heap[pos * kThreads + tid] = key;
+    tau = from_order_bits((uint32_t)(heap[tid] >> 32));
   };
   auto flush = [&]() {
     for (int e = 0; e < cnt; ++e) {
@@ -330,31 +299,35 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   }
 
   if (row_ok) {
-    // Kept past blocks: compact the live slots holding a real score, note the
-    // best score, sort the block indices ascending.
-    int kept = 0;
+    // Kept past blocks: the live heap slots holding a real key.  Note the
+    // best score, turn each slot into its block index (others into INT_MAX)
+    // and insertion-sort the indices ascending in place.
     float best = -INFINITY;
+    int kept = 0;
     for (int sl = 0; sl < k1; ++sl) {
-      const float v = lv[sl * kThreads + tid];
-      if (v > -INFINITY) {
-        best = fmaxf(best, v);
-        li[kept * kThreads + tid] = li[sl * kThreads + tid];
+      const uint64_t key = heap[sl * kThreads + tid];
+      int jj = 0x7fffffff;
+      if (key != kKeyEmpty) {
+        best = fmaxf(best, from_order_bits((uint32_t)(key >> 32)));
+        jj = (int)(0xffffffffu - (uint32_t)(key & 0xffffffffu));
         ++kept;
       }
+      heap[sl * kThreads + tid] = (uint64_t)(uint32_t)jj;
     }
-    for (int a = 1; a < kept; ++a) {
-      const int x = li[a * kThreads + tid];
+    for (int a = 1; a < k1; ++a) {
+      const uint64_t x = heap[a * kThreads + tid];
       int b2 = a - 1;
-      while (b2 >= 0 && li[b2 * kThreads + tid] > x) {
-        li[(b2 + 1) * kThreads + tid] = li[b2 * kThreads + tid];
+      while (b2 >= 0 && heap[b2 * kThreads + tid] > x) {
+        heap[(b2 + 1) * kThreads + tid] = heap[b2 * kThreads + tid];
         --b2;
       }
-      li[(b2 + 1) * kThreads + tid] = x;
+      heap[(b2 + 1) * kThreads + tid] = x;
     }
     const int t = t0 + tid;
     const size_t row = (size_t)t * h_q + h;
     int32_t* out = sel_idx + row * topk;
-    for (int m = 0; m < topk; ++m) out[m] = m < kept ? li[m * kThreads + tid] : (m == kept ? my_b : -1);
+    for (int m = 0; m < topk; ++m)
+      out[m] = m < kept ? (int32_t)heap[m * kThreads + tid] : (m == kept ? my_b : -1);
     const bf16* qrow = q + (size_t)t * qstride + (size_t)h * D;
     const bf16* krow = k + ((size_t)t * h_kv + kvh) * D;
     float dot = 0.f;
