@@ -46,7 +46,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch of each kernel, read from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
 # kernel source file it was taken with: a changed source voids the figure.
-NCU_TRAFFIC = {}
+# Headline workload, one timed-step launch each (profiles/dram_traffic_n64k_h16_d64_b32_k32_kconv4.md).
+NCU_TRAFFIC = {
+    "fwd_route": {"bytes": 296.89e6 + 405.32e6, "sha": "fa694e2b2a570312"},
+    "fwd_attn": {"bytes": 1.02e9 + 668.09e6, "sha": "c12b24e4d39fbab2"},
+    "bwd_attn": {"bytes": 1.11e9 + 590.14e6, "sha": "860c3246646589a8"},
+}
 
 
 # ----------------------------------------------------------------------------- helpers
