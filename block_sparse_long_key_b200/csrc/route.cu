@@ -13,8 +13,9 @@
 // ascending and padded with -1.
 //
 // One CTA owns 128 consecutive queries of one sequence and one query head.
-// Their Q tile and a stream of centroid chunks (NC blocks each, double
-// buffered, cp.async into 128-byte-swizzled K-major shared memory) feed
+// Their Q tile sits in tensor memory (thread t writes row t, the MMA's A
+// operand); a stream of centroid chunks (NC blocks each, double buffered,
+// cp.async into 128-byte-swizzled K-major shared memory) is the B operand of
 // tcgen05.mma (M = 128 queries, N = NC blocks, bf16 in, fp32 accumulate into
 // tensor memory, double buffered): one thread issues q.c_hi + q.c_lo, which
 // carries ~16 mantissa bits of the fp32 centroid, while the CTA's 128 threads
@@ -50,11 +51,9 @@ constexpr uint32_t kFull = 0xffffffffu;
 
 template <int D, int NC, int LISTN>
 struct RouteLayout {
-  static constexpr int kBuf = D == 64 ? 16 : 12;          // candidate buffer slots per thread
+  static constexpr int kBuf = 6;                          // candidate buffer slots per thread
   static constexpr int KB = D / 64;                       // 128-byte K blocks
-  static constexpr uint32_t Q_OFF = 0;
-  static constexpr uint32_t Q_REGION = kTM * 128;
-  static constexpr uint32_t C_OFF = Q_OFF + KB * Q_REGION;
+  static constexpr uint32_t C_OFF = 0;
   static constexpr uint32_t C_REGION = NC * 128;
   static constexpr uint32_t C_MAT = KB * C_REGION;       // hi or lo of one chunk
   static constexpr uint32_t C_BUF = 2 * C_MAT;           // hi + lo
@@ -62,13 +61,14 @@ struct RouteLayout {
   static constexpr uint32_t BV_OFF = HP_OFF + LISTN * kThreads * 8;
   static constexpr uint32_t BI_OFF = BV_OFF + kBuf * kThreads * 4;
   static constexpr uint32_t MB_OFF = BI_OFF + kBuf * kThreads * 4;
-  static_assert((LISTN & (LISTN - 1)) == 0, "heap is a complete tree of LISTN - 1 nodes");
   static constexpr uint32_t HOLD_OFF = MB_OFF + 16;
-  static constexpr uint32_t FLAG_OFF = HOLD_OFF + 4;
-  static constexpr uint32_t BYTES = FLAG_OFF + 12;
-  static constexpr uint32_t TMEM_COLS = 2 * NC;
-  static_assert(C_REGION % 1024 == 0 && Q_REGION % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
-  static_assert(TMEM_COLS >= 32 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation is a power of two");
+  static constexpr uint32_t BYTES = HOLD_OFF + 16;
+  // Tensor memory: two NC-column score tiles, then Q (D bf16 = D/2 columns).
+  static constexpr uint32_t TM_Q = 2 * NC;
+  static constexpr uint32_t TMEM_COLS = 128;
+  static_assert((LISTN & (LISTN - 1)) == 0, "heap is a complete tree of LISTN - 1 nodes");
+  static_assert(C_REGION % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
+  static_assert(TM_Q + D / 2 <= TMEM_COLS, "score tiles and Q fit the allocation");
 };
 
 __device__ __forceinline__ uint32_t order_bits(float v) {
@@ -117,13 +117,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   const int tid = threadIdx.x, warp = tid >> 5;
   const size_t qstride = (size_t)h_q * D;
 
-  // ---- loads: Q tile, centroid chunks (hi, lo), all into SW128 K-major layout
-  for (int i = tid; i < kTM * (D / 8); i += kThreads) {
-    const int r = i / (D / 8), cc = i % (D / 8);
-    const bool ok = r < nrows;
-    const size_t src = ok ? (size_t)(t0 + r) * qstride + (size_t)h * D + cc * 8 : 0;
-    cp_async16_zfill(sm + Ly::Q_OFF + (cc >> 3) * Ly::Q_REGION + tc::sw128_offset(r, cc & 7), q + src, ok);
-  }
+  // ---- loads: centroid chunks (hi, lo) into SW128 K-major layout
   const size_t head0 = ((size_t)kvh * nb_max + cbase) * D;
   auto load_chunk = [&](int c, int buf) {
     for (int i = tid; i < 2 * NC * (D / 8); i += kThreads) {
@@ -170,6 +164,25 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   tc::fence_after_sync();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
   constexpr uint32_t idesc = tc::idesc_bf16_f32(kTM, NC);
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  if (nchunks > 0) {
+    // Q row `tid` -> TMEM lane `tid`, columns TM_Q .. TM_Q + D/2 (bf16 pairs).
+    const bf16* qrow = q + (size_t)(t0 + tid) * qstride + (size_t)h * D;
+#pragma unroll
+    for (int half = 0; half < D / 64; ++half) {
+      uint32_t w[32];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 u = row_ok ? __ldg(reinterpret_cast<const uint4*>(qrow + half * 64 + c * 8)) : make_uint4(0, 0, 0, 0);
+        w[4 * c] = u.x;
+        w[4 * c + 1] = u.y;
+        w[4 * c + 2] = u.z;
+        w[4 * c + 3] = u.w;
+      }
+      tc::tmem_st32(tmem + lane_base + Ly::TM_Q + half * 32, w);
+    }
+    tc::tmem_st_wait();
+  }
 
   // Admit (x, j), x > tau: replace the root and sift it down.  Candidates
   // arrive in ascending j, so a score equal to the threshold never displaces
@@ -205,18 +218,18 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
 
   auto select_chunk = [&](int c, int buf) {
     uint32_t v[NC];
-    const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(buf * NC);
+    const uint32_t taddr = tmem + lane_base + (uint32_t)(buf * NC);
 #pragma unroll
     for (int hf = 0; hf < NC / 32; ++hf)
       tc::tmem_ld32(taddr + hf * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[hf * 32]));
     tc::tmem_ld_wait();
     const int jbase = c * NC;
 #pragma unroll
-    for (int g = 0; g < NC / 8; ++g) {
-      if (__any_sync(kFull, cnt > Ly::kBuf - 8)) flush();  // room for the next 8 columns
+    for (int g = 0; g < NC / 4; ++g) {
+      if (__any_sync(kFull, cnt > Ly::kBuf - 4)) flush();  // room for the next 4 columns
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int col = g * 8 + e;
+      for (int e = 0; e < 4; ++e) {
+        const int col = g * 4 + e;
         const float x = __uint_as_float(v[col]);
         const int j = jbase + col;
         if (j < my_b && x > tau) {
@@ -241,19 +254,18 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
     if (tid == 0) {
       tc::fence_after_sync();
       const uint32_t d_tmem = tmem + (uint32_t)(buf * NC);
-      const uint32_t qa = sbase + Ly::Q_OFF;
+      const uint32_t qa = tmem + Ly::TM_Q;  // lane 0, Q columns
       const uint32_t ca = sbase + Ly::C_OFF + buf * Ly::C_BUF;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t koff = (kk & 3) * 32;  // 16 bf16 per K step inside a 128-byte row
-        const uint64_t a = tc::sw128_desc(qa + (kk >> 2) * Ly::Q_REGION + koff);
-        tc::mma_bf16_ss(d_tmem, a, tc::sw128_desc(ca + (kk >> 2) * Ly::C_REGION + koff), idesc, kk > 0);
+        tc::mma_bf16_ts(d_tmem, qa + kk * 8, tc::sw128_desc(ca + (kk >> 2) * Ly::C_REGION + koff), idesc, kk > 0);
       }
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t koff = (kk & 3) * 32;
-        const uint64_t a = tc::sw128_desc(qa + (kk >> 2) * Ly::Q_REGION + koff);
-        tc::mma_bf16_ss(d_tmem, a, tc::sw128_desc(ca + Ly::C_MAT + (kk >> 2) * Ly::C_REGION + koff), idesc, 1u);
+        tc::mma_bf16_ts(d_tmem, qa + kk * 8, tc::sw128_desc(ca + Ly::C_MAT + (kk >> 2) * Ly::C_REGION + koff), idesc,
+                        1u);
       }
       tc::mma_commit(mbar0 + 8 * buf);
     }
@@ -369,8 +381,8 @@ cudaError_t launch_route(const bf16* q, const bf16* k, const bf16* hi, const bf1
 #define MOBA_ROUTE(DD, NCC, LN) \
   return launch_route_t<DD, NCC, LN>(q, k, hi, lo, p, h_q, h_kv, block_size, topk, sel, mref, flag, oacc, status, st)
   if (d == 64) {
-    if (k1 <= 32) MOBA_ROUTE(64, 64, 32);
-    MOBA_ROUTE(64, 64, 64);
+    if (k1 <= 32) MOBA_ROUTE(64, 32, 32);
+    MOBA_ROUTE(64, 32, 64);
   } else {
     if (k1 <= 32) MOBA_ROUTE(128, 32, 32);
     MOBA_ROUTE(128, 32, 64);
