@@ -63,6 +63,7 @@ __all__ = [
     "backward_rows",
     "block_selected_by",
     "block_index",
+    "key_conv_backward",
 ]
 
 # Largest finite bf16 value, (2 - 2^-7) * 2^127.
@@ -95,7 +96,7 @@ def _seqs(cu_seqlens) -> List[Tuple[int, int]]:
     return [(cu[s], cu[s + 1]) for s in range(len(cu) - 1)]
 
 
-def key_conv(k: np.ndarray, w: np.ndarray, cu_seqlens) -> np.ndarray:
+def key_conv(k: np.ndarray, w: np.ndarray, cu_seqlens, round_output: bool = True) -> np.ndarray:
     """Depthwise causal short convolution on keys, then bf16 rounding.
 
     Follows §"Progettazione della Convoluzione delle Chiavi (Appendice B)",
@@ -104,7 +105,8 @@ def key_conv(k: np.ndarray, w: np.ndarray, cu_seqlens) -> np.ndarray:
     before the sequence start contributes nothing.
 
     k: [T, H, d] float64 values of the bf16 keys.  w: [H, d, W] (tap l
-    multiplies k_{t-l}).  Returns k' as float64 values of bf16 numbers.
+    multiplies k_{t-l}).  Returns k' as float64 values of bf16 numbers
+    (``round_output=False``: the unrounded float64 values).
     """
     k = np.asarray(k, dtype=np.float64)
     w = np.asarray(w, dtype=np.float64)
@@ -119,7 +121,7 @@ def key_conv(k: np.ndarray, w: np.ndarray, cu_seqlens) -> np.ndarray:
                 shifted[l:] = ks[: ks.shape[0] - l]
             acc += w[None, :, :, l] * shifted
         out[a:b] = ks + silu(acc)
-    return round_bf16(out)
+    return round_bf16(out) if round_output else out
 
 
 def block_centroids(k: np.ndarray, cu_seqlens, block_size: int) -> List[np.ndarray]:
@@ -393,3 +395,41 @@ def block_index(sel, cu_seqlens, block_size: int, h_kv: int):
                         out.setdefault((h // g, off + int(j)), []).append(t * hq + h)
         off += (b - a + block_size - 1) // block_size
     return {key: sorted(v) for key, v in out.items()}
+
+
+def key_conv_backward(k: np.ndarray, w: np.ndarray, cu_seqlens, dk_conv: np.ndarray):
+    """Gradients of the key convolution: (dK, dW) from dK' = dL/dk'.
+
+    Differentiates the formula of ``key_conv`` (the final bf16 rounding is
+    treated as the identity): with x_t = sum_l W_l (.) k_{t-l} and
+    g_t = dK'_t (.) SiLU'(x_t), SiLU'(x) = s(x) (1 + x (1 - s(x))), s the
+    logistic function:
+      dK_t = dK'_t + sum_l W_l (.) g_{t+l}      (t + l inside the sequence)
+      dW_l = sum_t g_t (.) k_{t-l}              (summed over all sequences)
+    k, dk_conv: [T, H, d]; w: [H, d, W].  Returns dK [T, H, d], dW [H, d, W].
+    """
+    k = np.asarray(k, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    g_in = np.asarray(dk_conv, dtype=np.float64)
+    width = w.shape[2]
+    dk = g_in.copy()
+    dw = np.zeros_like(w)
+    for a, b in _seqs(cu_seqlens):
+        ks = k[a:b]
+        L = ks.shape[0]
+        x = np.zeros_like(ks)
+        shifted = []
+        for l in range(width):
+            sh = np.zeros_like(ks)
+            if l < L:
+                sh[l:] = ks[: L - l]
+            shifted.append(sh)
+            x += w[None, :, :, l] * sh
+        sig = 1.0 / (1.0 + np.exp(-x))
+        g = g_in[a:b] * sig * (1.0 + x * (1.0 - sig))
+        for l in range(width):
+            # dK_t gains W_l g_{t+l}; dW_l gains g_t k_{t-l}
+            if l < L:
+                dk[a:b][: L - l] += w[None, :, :, l] * g[l:]
+            dw[:, :, l] += (g * shifted[l]).sum(axis=0)
+    return dk, dw

@@ -379,3 +379,52 @@ def test_block_index_is_a_partition_of_the_picks():
             for j in sel[t, h]:
                 if j >= 0:
                     assert t * hq + h in idx[(h // 2, offs[s] + int(j))]
+
+
+# ---------------------------------------------------------------- key conv backward
+
+def test_key_conv_backward_matches_finite_differences():
+    r = _rng(16)
+    cu = [0, 7, 12]
+    T, H, d, W = 12, 2, 3, 3
+    k = r.standard_normal((T, H, d))
+    w = r.uniform(-0.5, 0.5, (H, d, W))
+    g = r.standard_normal((T, H, d))
+    dk, dw = orc.key_conv_backward(k, w, cu, g)
+    loss = lambda kk, ww: float((orc.key_conv(kk, ww, cu, round_output=False) * g).sum())
+    eps = 1e-6
+    for name, x, grad in (("k", k, dk), ("w", w, dw)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[i] += eps
+            xm[i] -= eps
+            lp = loss(xp, w) if name == "k" else loss(k, xp)
+            lm = loss(xm, w) if name == "k" else loss(k, xm)
+            num[i] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8, err_msg=name)
+
+
+def test_key_conv_backward_matches_library_autograd():
+    r = _rng(17)
+    cu = [0, 20, 20, 45]
+    T, H, d, W = 45, 2, 4, 4
+    k = r.standard_normal((T, H, d))
+    w = r.uniform(-0.5, 0.5, (H, d, W))
+    g = r.standard_normal((T, H, d))
+    dk, dw = orc.key_conv_backward(k, w, cu, g)
+    tk = torch.tensor(k, requires_grad=True)
+    tw = torch.tensor(w, requires_grad=True)
+    outs = []
+    for a, b in zip(cu[:-1], cu[1:]):
+        if a == b:
+            continue   # an empty sequence contributes nothing
+        x = tk[a:b].reshape(b - a, H * d).T[None]
+        wt = tw.flip(-1).reshape(H * d, 1, W)
+        y = F.conv1d(F.pad(x, (W - 1, 0)), wt, groups=H * d)[0].T.reshape(b - a, H, d)
+        outs.append(tk[a:b] + F.silu(y))
+    torch.cat(outs).backward(torch.tensor(g))
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dw, tw.grad.numpy(), rtol=1e-12, atol=1e-12)
