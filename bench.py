@@ -173,17 +173,21 @@ def stage_roofline(name, w, pairs, scored, peaks):
         return "hbm", T * hq * d * 6.0, "byte"
     if name in ("fwd_index", "bwd_index"):
         return "hbm", T * hq * w.topk * 4.0 * 2 + pairs * 4.0 * 3, "byte"
+    if name == "conv_bwd":
+        return "hbm", T * hkv * d * 2.0 * 3, "byte"
     return "hbm", 0.0, "byte"
 
 
 KERNEL_SRC = {"fwd_attn": "fwd.cu", "bwd_attn": "bwd.cu", "fwd_route": "route.cu", "fwd_centroid": "conv_centroid.cu",
               "fwd_finalize": "fwd.cu", "bwd_pre": "bwd.cu", "bwd_dq": "bwd.cu", "fwd_index": "index.cu",
-              "bwd_index": "index.cu"}
+              "bwd_index": "index.cu", "conv_bwd": "conv_bwd.cu"}
 
 # Kernels of ours launched per step: forward 10 (plan, conv/centroid, route,
 # index count, prefix, scan, fill, attention, finalize, fallback), backward 4
-# (plan, preprocess, attention, dQ; the forward's block index is reused).
+# (plan, preprocess, attention, dQ; the forward's block index is reused),
+# key-conv backward 3 (plan, per-block pass, dW reduction) when the conv is on.
 LAUNCHES_PER_STEP = 14
+LAUNCHES_CONV_BWD = 3
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) timing
@@ -263,12 +267,16 @@ def run_ours(args):
     kc = torch.empty_like(g["k"]) if w.conv_width else None
     dq, dk, dv = torch.empty_like(g["q"]), torch.empty_like(g["k"]), torch.empty_like(g["v"])
     conv_w = g.get("conv_w")
+    dk_in = torch.empty_like(g["k"]) if conv_w is not None else None
+    dw = torch.empty_like(conv_w) if conv_w is not None else None
 
     def step(qd, kd, vd, dod, cud, cw):
         _, _, _, k_used = moba.forward(qd, kd, vd, cud, B, topk, conv_w=cw, workspace=ws_f, out=out, lse=lse,
                                        sel_idx=sel, k_conv=kc)
         moba.backward(qd, k_used, vd, out, lse, dod, sel, cud, B, workspace=ws_b, dq=dq, dk=dk, dv=dv,
                       fwd_workspace=ws_f)
+        if cw is not None:   # through the key conv: gradients of the original keys and of the weights
+            moba.key_conv_backward(kd, cw, cud, B, dk, workspace=ws_b, dk=dk_in, dw=dw)
 
     for _ in range(args.warmup):
         step(g["q"], g["k"], g["v"], g["dout"], g["cu_seqlens"], conv_w)
@@ -301,7 +309,7 @@ def run_ours(args):
     for s in moba.STAGES:
         stage_ms[s] = statistics.mean(e.ms()[s] for e in stage_sets)
     fwd_ms = sum(v for k_, v in stage_ms.items() if k_.startswith("fwd"))
-    bwd_ms = sum(v for k_, v in stage_ms.items() if k_.startswith("bwd"))
+    bwd_ms = sum(v for k_, v in stage_ms.items() if k_.startswith("bwd") or k_ == "conv_bwd")
 
     flops = w.fwd_flops() + w.bwd_flops()
     value = aggregate_value(flops, world, ms_max)
@@ -330,7 +338,7 @@ def run_ours(args):
         names_in = ["q", "k", "v", "dout"] + (["conv_w"] if conv_w is not None else []) + ["cu_seqlens"]
         host = {n: x[n].pin_memory() for n in names_in}
         dev_in = {n: torch.empty_like(g[n]) for n in names_in}
-        outs = [out, lse, dq, dk, dv]
+        outs = [out, lse, dq, dk, dv] + ([dk_in, dw] if conv_w is not None else [])
         host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = sum(t.numel() * t.element_size() for t in outs)
@@ -383,7 +391,7 @@ def run_ours(args):
             "peak_bf16_tflops": peak_t, "peak_source": peak_src,
             "stage_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
             "pairs": pairs, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks.summary(), "device_status": status,
+            "gpu_launches": (LAUNCHES_PER_STEP + (LAUNCHES_CONV_BWD if w.conv_width else 0)) * args.steps, "clocks": clocks.summary(), "device_status": status,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -51,6 +51,7 @@ conv_centroid_kernel(const bf16* __restrict__ k, const float* __restrict__ conv_
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 
   if (width == 0) {
+#pragma unroll 4
     for (int t = t0; t < t1; ++t) {
       float f[8];
       bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kh + (size_t)t * row_stride)), f);
@@ -77,6 +78,7 @@ conv_centroid_kernel(const bf16* __restrict__ k, const float* __restrict__ conv_
       }
     }
     bf16* ko = k_out + (size_t)h * D + c8 * 8;
+#pragma unroll 2
     for (int t = t0; t < t1; ++t) {
       float cur[8], x[8];
       bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kh + (size_t)t * row_stride)), cur);

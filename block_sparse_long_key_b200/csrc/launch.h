@@ -70,4 +70,9 @@ cudaError_t launch_bwd_attn(const bf16* q, const bf16* k, const bf16* v, const b
 
 cudaError_t launch_bwd_dq(const float* dqacc, int n, bf16* dq, cudaStream_t st);
 
+// dw_part: h_kv * nb_max * d * conv_width floats of per-block partial sums.
+cudaError_t launch_conv_bwd(const bf16* k, const float* conv_w, int conv_width, const bf16* dk_conv,
+                            const SeqPlan& p, int h_kv, int d, int block_size, bf16* dk, float* dw,
+                            float* dw_part, cudaStream_t st);
+
 }  // namespace moba

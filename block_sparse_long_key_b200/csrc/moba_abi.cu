@@ -107,6 +107,7 @@ struct BwdBufs {
   int32_t* chunk_cnt;
   float* dsum;
   float* dqacc;
+  float* dw_part;  // per-block key-conv dW partials (width <= 8)
 };
 
 BwdBufs carve_bwd(Carve& c, const moba_shape* s) {
@@ -122,6 +123,7 @@ BwdBufs carve_bwd(Carve& c, const moba_shape* s) {
   b.chunk_cnt = nch ? c.take<int32_t>(nch) : nullptr;
   b.dsum = c.take<float>(nrow);
   b.dqacc = c.take<float>(nrow * s->head_dim);
+  b.dw_part = c.take<float>((size_t)s->h_kv * nb_max_of(s) * s->head_dim * 8);
   return b;
 }
 
@@ -131,8 +133,10 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 thread_local cudaEvent_t const* g_stage_events = nullptr;
 thread_local int g_stage_nevents = 0;
 
+// idx < 0 (a plan run by a step entry point without a stage of its own) is not recorded.
 void stage_mark(int idx, cudaStream_t st) {
-  if (g_stage_events && idx < g_stage_nevents && g_stage_events[idx]) cudaEventRecord(g_stage_events[idx], st);
+  if (g_stage_events && idx >= 0 && idx < g_stage_nevents && g_stage_events[idx])
+    cudaEventRecord(g_stage_events[idx], st);
 }
 #define STAGE_BEGIN(i) stage_mark(2 * (i), st)
 #define STAGE_END(i) stage_mark(2 * (i) + 1, st)
@@ -326,6 +330,30 @@ int moba_backward(const void* q, const void* k, const void* v, const void* out, 
   STAGE_BEGIN(MOBA_STAGE_BWD_DQ);
   MOBA_TRY(moba::launch_bwd_dq(b.dqacc, T * hq * d, static_cast<bf16*>(dq), st));
   STAGE_END(MOBA_STAGE_BWD_DQ);
+  return MOBA_OK;
+}
+
+int moba_key_conv_backward(const void* k, const float* conv_w, int conv_width, const int32_t* cu_seqlens,
+                           const moba_shape* shape, const void* dk_conv, void* dk, float* dw, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (!shape_ok(shape)) return MOBA_EINVAL;
+  if (conv_width < 1 || conv_width > 8) return MOBA_EINVAL;
+  if (shape->total_tokens == 0) return MOBA_OK;
+  int rc;
+  if ((rc = check_ptrs({k, conv_w, cu_seqlens, dk_conv, dk, dw})) != MOBA_OK) return rc;
+  if (dk == k || dk == dk_conv) return MOBA_EINVAL;
+  if ((rc = check_ws(workspace, workspace_bytes, moba_bwd_workspace_size(shape))) != MOBA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carve c;
+  c.base = static_cast<char*>(workspace);
+  BwdBufs b = carve_bwd(c, shape);
+  moba::SeqPlan plan;
+  if ((rc = begin_plan(b.plan, cu_seqlens, shape, st, &plan, -1)) != MOBA_OK) return rc;
+  STAGE_BEGIN(MOBA_STAGE_CONV_BWD);
+  MOBA_TRY(moba::launch_conv_bwd(static_cast<const bf16*>(k), conv_w, conv_width, static_cast<const bf16*>(dk_conv),
+                                 plan, shape->h_kv, shape->head_dim, shape->block_size, static_cast<bf16*>(dk), dw,
+                                 b.dw_part, st));
+  STAGE_END(MOBA_STAGE_CONV_BWD);
   return MOBA_OK;
 }
 

@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.moba_build_index.restype = I
         L.moba_backward.argtypes = [P, P, P, P, P, P, P, P, F, P, P, P, P, S, P, P]
         L.moba_backward.restype = I
+        L.moba_key_conv_backward.argtypes = [P, P, I, P, F, P, P, P, P, S, P]
+        L.moba_key_conv_backward.restype = I
         L.moba_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), I]
         L.moba_set_stage_events.restype = I
         L.moba_check_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
@@ -222,7 +224,7 @@ def backward(q, k, v, out, lse, dout, sel_idx, cu_seqlens, block_size: int, work
 
 
 STAGES = ["fwd_plan", "fwd_centroid", "fwd_route", "fwd_index", "fwd_attn", "fwd_finalize",
-          "bwd_plan", "bwd_index", "bwd_pre", "bwd_attn", "bwd_dq"]
+          "bwd_plan", "bwd_index", "bwd_pre", "bwd_attn", "bwd_dq", "conv_bwd"]
 
 
 class StageEvents:
@@ -244,6 +246,23 @@ class StageEvents:
 
     def ms(self):
         return {n: self.events[2 * i].elapsed_time(self.events[2 * i + 1]) for i, n in enumerate(STAGES)}
+
+
+def key_conv_backward(k, conv_w, cu_seqlens, block_size: int, dk_conv, workspace=None, dk=None, dw=None, h_q=None):
+    """Gradients of the key conv: (dK of the original keys, dW [h_kv, d, W])."""
+    _need(k, torch.bfloat16, "k", 3)
+    _need(dk_conv, torch.bfloat16, "dk_conv", 3)
+    _need(conv_w, torch.float32, "conv_w", 3)
+    _need(cu_seqlens, torch.int32, "cu_seqlens", 1)
+    T, hkv, d = k.shape
+    shape = make_shape(T, cu_seqlens.numel() - 1, h_q or hkv, hkv, d, block_size, 1)
+    dk = torch.empty_like(k) if dk is None else dk
+    dw = torch.empty_like(conv_w) if dw is None else dw
+    ws = workspace if workspace is not None else alloc_workspace(bwd_workspace_size(shape), k.device)
+    rc = lib().moba_key_conv_backward(_ptr(k), _ptr(conv_w), conv_w.shape[2], _ptr(cu_seqlens), ctypes.byref(shape),
+                                      _ptr(dk_conv), _ptr(dk), _ptr(dw), _ptr(ws), ws.numel(), _stream())
+    _check(rc, "moba_key_conv_backward")
+    return dk, dw
 
 
 def check_status(workspace: torch.Tensor) -> int:

@@ -84,6 +84,11 @@ def _randn_bf16(shape, seed, tensor_id) -> torch.Tensor:
     return torch.randn(shape, generator=_gen(seed, tensor_id), dtype=torch.float32).to(torch.bfloat16)
 
 
+def randn_bf16(shape, seed: int, tensor_id: int = 7) -> torch.Tensor:
+    """A seeded N(0, 1) bf16 tensor (e.g. an incoming gradient)."""
+    return _randn_bf16(tuple(shape), seed, tensor_id)
+
+
 def cu_seqlens_of(seqlens) -> torch.Tensor:
     cu = [0]
     for L in seqlens:

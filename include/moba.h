@@ -212,7 +212,8 @@ int moba_backward(const void* q, const void* k, const void* v, const void* out, 
  * for every i with 2*i+1 < n_events; NULL entries are skipped.  The stages:
  * forward plan, key conv + centroids, routing, block index, attention,
  * normalisation (+ exact re-computation of flagged rows); backward plan,
- * block index, preprocessing, attention, dQ conversion.  The table is read,
+ * block index, preprocessing, attention, dQ conversion; key-conv backward
+ * (moba_key_conv_backward).  The table is read,
  * never written; the caller keeps it (and the events) alive while installed.
  * Pass (NULL, 0) to remove it.  Results are unaffected.
  */
@@ -227,8 +228,30 @@ int moba_backward(const void* q, const void* k, const void* v, const void* out, 
 #define MOBA_STAGE_BWD_PRE 8
 #define MOBA_STAGE_BWD_ATTN 9
 #define MOBA_STAGE_BWD_DQ 10
-#define MOBA_NUM_STAGES 11
+#define MOBA_STAGE_CONV_BWD 11
+#define MOBA_NUM_STAGES 12
 int moba_set_stage_events(void* const* events, int n_events);
+
+/*
+ * Backward of the key convolution, for training with it: from dK' (the
+ * gradient moba_backward returns for k', which the attention used) to the
+ * gradient of the original keys and of the conv weights.  Differentiates
+ * "Optimizing Mixture of Block Attention", section "Progettazione della
+ * Convoluzione delle Chiavi (Appendice B)", "Forma Formale", with
+ * x_t = sum_l w_l (.) k_{t-l} and g_t = dK'_t (.) SiLU'(x_t):
+ *   dK_t = dK'_t + sum_l w_l (.) g_{t+l}   (t + l inside the sequence)
+ *   dW_l = sum_t g_t (.) k_{t-l}
+ * The bf16 rounding of k' is treated as the identity.
+ *
+ *  k, conv_w, conv_width, cu_seqlens   as given to moba_forward (1 <= width <= 8)
+ *  dk_conv   bf16 [T, h_kv, d]  dK' (e.g. moba_backward's dk)
+ *  dk        bf16 [T, h_kv, d]  output; must alias neither k nor dk_conv
+ *  dw        fp32 [h_kv, d, conv_width]  output (overwritten, not accumulated)
+ *  workspace >= moba_bwd_workspace_size(shape) bytes
+ */
+int moba_key_conv_backward(const void* k, const float* conv_w, int conv_width, const int32_t* cu_seqlens,
+                           const moba_shape* shape, const void* dk_conv, void* dk, float* dw, void* workspace,
+                           size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, then reads the status word the last call on this
  * workspace left.  *device_status receives the MOBA_STATUS_* bits (0 = ok).

@@ -93,3 +93,15 @@ def test_binding_refuses_cpu_tensors():
     cu = torch.tensor([0, 8], dtype=torch.int32)
     with pytest.raises(TypeError):
         moba.forward(q, q, q, cu, 16, 1)
+
+
+def test_stage_table_ignores_plans_without_a_stage(L):
+    # A fake, never-dereferenced table: entry points whose plan has no stage
+    # (index -1) must not read before its start.  Nothing runs on a device:
+    # the call stops at the workspace check.
+    arr = (ctypes.c_void_p * 4)(None, None, None, None)
+    assert L.moba_set_stage_events(arr, 4) == moba.MOBA_OK
+    s = _shape(total_tokens=1024, h_q=2, h_kv=1)
+    ok = ctypes.c_void_p(1 << 20)
+    assert L.moba_key_conv_centroid(ok, None, 0, ok, ctypes.byref(s), None, ok, ok, 16, None) == moba.MOBA_EWORKSPACE
+    assert L.moba_set_stage_events(None, 0) == moba.MOBA_OK

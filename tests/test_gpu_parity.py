@@ -255,3 +255,20 @@ def test_backward_reusing_forward_index_matches_oracle(dev, case):
     pu.check_grad(pu.to64(dq), dq_r, sq, "dq reuse")
     pu.check_grad(pu.to64(dk), dk_r, sk, "dk reuse")
     pu.check_grad(pu.to64(dv), dv_r, sv, "dv reuse")
+
+
+@pytest.mark.parametrize("case", [SMALL[3], SMALL[7], ((300, 5, 700), 2, 2, 128, 16, 4, 5)], ids=_ids)
+def test_key_conv_backward_matches_oracle(dev, case):
+    w, x = _inputs(case)
+    g = _gpu(x, dev)
+    dkc = synth.randn_bf16(x["k"].shape, seed=21)
+    dk, dw = moba.key_conv_backward(g["k"], g["conv_w"], g["cu_seqlens"], w.block_size, dkc.to(dev))
+    torch.cuda.synchronize()
+    dk_r, dw_r = orc.key_conv_backward(x["k"].double().numpy(), x["conv_w"].double().numpy(), x["cu_seqlens"].numpy(),
+                                       dkc.double().numpy())
+    # dK: fp32 arithmetic, then one bf16 rounding (relative 2^-9 of the value).
+    err = np.abs(pu.to64(dk) - dk_r)
+    rms = np.sqrt((dk_r ** 2).mean())
+    assert np.all(err <= 2.0 ** -8 * np.abs(dk_r) + 1e-5 * rms), (err / (np.abs(dk_r) + rms)).max()
+    # dW: fp32 sums over every token of a head.
+    np.testing.assert_allclose(pu.to64(dw), dw_r, rtol=1e-3, atol=1e-4 * np.abs(dw_r).max())
