@@ -48,9 +48,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel source file it was taken with: a changed source voids the figure.
 # Headline workload, one timed-step launch each (profiles/dram_traffic_n64k_h16_d64_b32_k32_kconv4.md).
 NCU_TRAFFIC = {
-    "fwd_route": {"bytes": 296.89e6 + 405.32e6, "sha": "fa694e2b2a570312"},
+    "fwd_route": {"bytes": 313.64e6 + 408.26e6, "sha": "6f9dfb1cc06a69b2"},
     "fwd_attn": {"bytes": 1.02e9 + 668.09e6, "sha": "c12b24e4d39fbab2"},
-    "bwd_attn": {"bytes": 1.11e9 + 590.14e6, "sha": "860c3246646589a8"},
+    "bwd_attn": {"bytes": 1.11e9 + 591.03e6, "sha": "860c3246646589a8"},
+    "conv_bwd": {"bytes": 269.38e6 + 131.24e6, "sha": "5f8d17997de2fc78"},
 }
 
 
