@@ -79,6 +79,38 @@ __device__ __forceinline__ float from_order_bits(uint32_t u) {
   return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
 }
 
+// One compare-exchange step of a bitonic network over the 32E keys a warp
+// holds (key i = lane * E + e): key i is paired with key i ^ j, and a block
+// of k keys is ordered descending where (i & k) == 0, ascending elsewhere.
+template <int E>
+__device__ __forceinline__ void bitonic_step(uint64_t (&x)[E], int lane, int k, int j) {
+  if (j < E) {  // E == 2, j == 1: both keys of the lane, same block direction
+    const bool desc = ((lane * E) & k) == 0;
+    const uint64_t hi = x[0] > x[E - 1] ? x[0] : x[E - 1];
+    const uint64_t lo = x[0] > x[E - 1] ? x[E - 1] : x[0];
+    x[0] = desc ? hi : lo;
+    x[E - 1] = desc ? lo : hi;
+  } else {
+    const int jl = j / E;
+    const bool lower = (lane & jl) == 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const uint64_t p = __shfl_xor_sync(kFull, x[e], jl);
+      const bool desc = ((lane * E + e) & k) == 0;
+      x[e] = (x[e] > p) == (lower == desc) ? x[e] : p;
+    }
+  }
+}
+
+// Sorts the warp's 32E keys descending (key i at lane i / E, slot i % E).
+template <int E>
+__device__ __forceinline__ void warp_sort_desc(uint64_t (&x)[E], int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32 * E; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) bitonic_step<E>(x, lane, k, j);
+}
+
 template <int D, int NC, int LISTN>
 __global__ void __launch_bounds__(kThreads)
 route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ cent_hi,
@@ -114,7 +146,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   const int k1 = topk - 1;
   const int nscan = k1 > 0 ? (p0 + nrows - 1) / block_size : 0;  // blocks any row may score
   const int nchunks = (nscan + NC - 1) / NC;
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t qstride = (size_t)h_q * D;
 
   // ---- loads: centroid chunks (hi, lo) into SW128 K-major layout
@@ -191,6 +223,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
     const uint64_t key = ((uint64_t)order_bits(x) << 32) | (uint64_t)(0xffffffffu - (uint32_t)j);
     int pos = 0;
     bool done = false;
+    uint64_t root = key;  // the new minimum: the key itself or the smaller child of the root
 #pragma unroll
     for (int lvl = 0; lvl < kHeapDepth; ++lvl) {
       const int c1 = 2 * pos + 1;
@@ -200,13 +233,14 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
       const uint64_t km = left ? k1v : k2v;
       if (!done && km < key) {
         heap[pos * kThreads + tid] = km;
+        if (lvl == 0) root = km;
         pos = left ? c1 : c1 + 1;
       } else {
         done = true;
       }
     }
     heap[pos * kThreads + tid] = key;
-    tau = from_order_bits((uint32_t)(heap[tid] >> 32));
+    tau = from_order_bits((uint32_t)(root >> 32));
   };
   auto flush = [&]() {
     for (int e = 0; e < cnt; ++e) {
@@ -310,36 +344,44 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
     tc::tmem_dealloc(tmem, Ly::TMEM_COLS);
   }
 
+  // One row at a time per warp: the kept keys (live heap slots holding a
+  // real key) become block indices, sorted ascending across the lanes and
+  // written coalesced, followed by the own block and -1 padding.
+  constexpr int E = LISTN / 32;
+  float best_mine = -INFINITY;
+  const int rows_here = min(32, nrows - warp * 32);
+  for (int r = 0; r < rows_here; ++r) {
+    const int rr = warp * 32 + r;
+    uint64_t y[E], top = 0ull;
+    int kept_n = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int i = lane * E + e;
+      const uint64_t key = i < k1 ? heap[i * kThreads + rr] : kKeyEmpty;
+      const bool real = key != kKeyEmpty;
+      kept_n += __popc(__ballot_sync(kFull, real));
+      y[e] = real ? (key & 0xffffffffull) : 0ull;  // inverted index: larger = lower block
+      top = real && key > top ? key : top;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const uint64_t o = __shfl_xor_sync(kFull, top, off);
+      top = o > top ? o : top;
+    }
+    if (lane == r && top) best_mine = from_order_bits((uint32_t)(top >> 32));
+    warp_sort_desc<E>(y, lane);
+    const int own = __shfl_sync(kFull, my_b, r);
+    int32_t* out = sel_idx + ((size_t)(t0 + rr) * h_q + h) * topk;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int i = lane * E + e;
+      if (i < topk) out[i] = i < kept_n ? (int32_t)(0xffffffffu - (uint32_t)y[e]) : (i == kept_n ? own : -1);
+    }
+  }
+
   if (row_ok) {
-    // Kept past blocks: the live heap slots holding a real key.  Note the
-    // best score, turn each slot into its block index (others into INT_MAX)
-    // and insertion-sort the indices ascending in place.
-    float best = -INFINITY;
-    int kept = 0;
-    for (int sl = 0; sl < k1; ++sl) {
-      const uint64_t key = heap[sl * kThreads + tid];
-      int jj = 0x7fffffff;
-      if (key != kKeyEmpty) {
-        best = fmaxf(best, from_order_bits((uint32_t)(key >> 32)));
-        jj = (int)(0xffffffffu - (uint32_t)(key & 0xffffffffu));
-        ++kept;
-      }
-      heap[sl * kThreads + tid] = (uint64_t)(uint32_t)jj;
-    }
-    for (int a = 1; a < k1; ++a) {
-      const uint64_t x = heap[a * kThreads + tid];
-      int b2 = a - 1;
-      while (b2 >= 0 && heap[b2 * kThreads + tid] > x) {
-        heap[(b2 + 1) * kThreads + tid] = heap[b2 * kThreads + tid];
-        --b2;
-      }
-      heap[(b2 + 1) * kThreads + tid] = x;
-    }
     const int t = t0 + tid;
     const size_t row = (size_t)t * h_q + h;
-    int32_t* out = sel_idx + row * topk;
-    for (int m = 0; m < topk; ++m)
-      out[m] = m < kept ? (int32_t)heap[m * kThreads + tid] : (m == kept ? my_b : -1);
     const bf16* qrow = q + (size_t)t * qstride + (size_t)h * D;
     const bf16* krow = k + ((size_t)t * h_kv + kvh) * D;
     float dot = 0.f;
@@ -351,7 +393,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
 #pragma unroll
       for (int i = 0; i < 8; ++i) dot = fmaf(fq[i], fk[i], dot);
     }
-    mref[row] = fmaxf(best, dot) * rsqrtf((float)D);
+    mref[row] = fmaxf(best_mine, dot) * rsqrtf((float)D);
     flag[row] = 0;
   }
 }
