@@ -48,6 +48,7 @@ constexpr uint64_t kKeyMax = ~0ull;  // heap padding: never the minimum
 // the root's score reads back as -inf until k-1 blocks have been admitted.
 constexpr uint64_t kKeyEmpty = (uint64_t)0x007fffffu << 32;
 constexpr uint32_t kFull = 0xffffffffu;
+constexpr int kGroup = 4;  // columns appended between buffer checks
 
 template <int D, int NC, int LISTN>
 struct RouteLayout {
@@ -58,9 +59,8 @@ struct RouteLayout {
   static constexpr uint32_t C_MAT = KB * C_REGION;       // hi or lo of one chunk
   static constexpr uint32_t C_BUF = 2 * C_MAT;           // hi + lo
   static constexpr uint32_t HP_OFF = C_OFF + 2 * C_BUF;           // heap keys [LISTN][kThreads] u64
-  static constexpr uint32_t BV_OFF = HP_OFF + LISTN * kThreads * 8;
-  static constexpr uint32_t BI_OFF = BV_OFF + kBuf * kThreads * 4;
-  static constexpr uint32_t MB_OFF = BI_OFF + kBuf * kThreads * 4;
+  static constexpr uint32_t BK_OFF = HP_OFF + LISTN * kThreads * 8;  // candidate keys [kBuf][kThreads] u64
+  static constexpr uint32_t MB_OFF = BK_OFF + kBuf * kThreads * 8;
   static constexpr uint32_t HOLD_OFF = MB_OFF + 16;
   static constexpr uint32_t BYTES = HOLD_OFF + 16;
   // Tensor memory: two NC-column score tiles, then Q (D bf16 = D/2 columns).
@@ -77,6 +77,10 @@ __device__ __forceinline__ uint32_t order_bits(float v) {
 }
 __device__ __forceinline__ float from_order_bits(uint32_t u) {
   return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+// Larger key = better block: higher score, then lower index.
+__device__ __forceinline__ uint64_t make_key(float x, int j) {
+  return ((uint64_t)order_bits(x) << 32) | (uint64_t)(0xffffffffu - (uint32_t)j);
 }
 
 // One compare-exchange step of a bitonic network over the 32E keys a warp
@@ -127,8 +131,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(sm);
   uint64_t* heap = reinterpret_cast<uint64_t*>(sm + Ly::HP_OFF);
-  float* bv = reinterpret_cast<float*>(sm + Ly::BV_OFF);
-  int32_t* bi = reinterpret_cast<int32_t*>(sm + Ly::BI_OFF);
+  uint64_t* bk = reinterpret_cast<uint64_t*>(sm + Ly::BK_OFF);
   const uint32_t mbar0 = sbase + Ly::MB_OFF;
 
   const int ntiles = __ldg(tile_off + batch);
@@ -175,8 +178,9 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   // Min-heap of the kept keys: k1 live slots start empty (score -inf),
   // padding slots up to LISTN-1 hold kKeyMax and never surface.
   for (int sl = 0; sl < LISTN; ++sl) heap[sl * kThreads + tid] = sl < k1 ? kKeyEmpty : kKeyMax;
-  float tau = -INFINITY;  // score of the root (the worst kept entry)
-  int cnt = 0;
+  uint64_t root_key = kKeyEmpty;  // the heap's root: the worst kept key
+  float tau = -INFINITY;          // its score
+  int cnt = 0;                    // buffered candidate keys
   if (tid == 0) {
     tc::mbar_init(mbar0, 1);
     tc::mbar_init(mbar0 + 8, 1);
@@ -216,11 +220,8 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
     tc::tmem_st_wait();
   }
 
-  // Admit (x, j), x > tau: replace the root and sift it down.  Candidates
-  // arrive in ascending j, so a score equal to the threshold never displaces
-  // it (lower index wins ties): the strict test on the score is exact.
-  auto admit = [&](float x, int j) {
-    const uint64_t key = ((uint64_t)order_bits(x) << 32) | (uint64_t)(0xffffffffu - (uint32_t)j);
+  // Admit a key above the root: replace the root and sift it down.
+  auto admit = [&](uint64_t key) {
     int pos = 0;
     bool done = false;
     uint64_t root = key;  // the new minimum: the key itself or the smaller child of the root
@@ -240,14 +241,19 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
       }
     }
     heap[pos * kThreads + tid] = key;
+    root_key = root;
     tau = from_order_bits((uint32_t)(root >> 32));
   };
-  auto flush = [&]() {
-    for (int e = 0; e < cnt; ++e) {
-      const float x = bv[e * kThreads + tid];
-      if (x > tau) admit(x, bi[e * kThreads + tid]);
+  // One round: every thread with buffered keys admits its latest one (full
+  // keys are compared, so the order of admission does not matter).  Rounds
+  // run only while some thread's buffer is close to full, so most threads
+  // have work in each of them.
+  auto flush_round = [&]() {
+    if (cnt > 0) {
+      --cnt;
+      const uint64_t key = bk[cnt * kThreads + tid];
+      if (key > root_key) admit(key);
     }
-    cnt = 0;
   };
 
   auto select_chunk = [&](int c, int buf) {
@@ -259,21 +265,18 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
     tc::tmem_ld_wait();
     const int jbase = c * NC;
 #pragma unroll
-    for (int g = 0; g < NC / 4; ++g) {
-      if (__any_sync(kFull, cnt > Ly::kBuf - 4)) flush();  // room for the next 4 columns
+    for (int g = 0; g < NC / kGroup; ++g) {
+      while (__any_sync(kFull, cnt > Ly::kBuf - kGroup)) flush_round();  // room for the next group
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int col = g * 4 + e;
+      for (int e = 0; e < kGroup; ++e) {
+        const int col = g * kGroup + e;
         const float x = __uint_as_float(v[col]);
         const int j = jbase + col;
-        if (j < my_b && x > tau) {
-          bv[cnt * kThreads + tid] = x;
-          bi[cnt * kThreads + tid] = j;
-          ++cnt;
-        }
+        // Blocks arrive in ascending j, so a score equal to tau (the root's,
+        // which has a lower index) never wins: the strict test is exact.
+        if (j < my_b && x > tau) bk[(cnt++) * kThreads + tid] = make_key(x, j);
       }
     }
-    if (__any_sync(kFull, cnt > 0)) flush();
   };
 
   // All waits are decided block-wide (__syncthreads_and), so every thread
@@ -323,6 +326,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
     if (__syncthreads_and(got)) {
       tc::fence_after_sync();
       select_chunk(pc, pc & 1);
+      while (__any_sync(kFull, cnt > 0)) flush_round();
     } else {
       ok = false;
     }
