@@ -179,7 +179,7 @@ def stage_roofline(name, w, pairs, scored, peaks):
     return "hbm", 0.0, "byte"
 
 
-KERNEL_SRC = {"fwd_attn": "fwd.cu", "bwd_attn": "bwd.cu", "fwd_route": "route.cu", "fwd_centroid": "conv_centroid.cu",
+KERNEL_SRC = {"fwd_attn": "fwd.cu", "bwd_attn": "bwd_tc.cu", "fwd_route": "route.cu", "fwd_centroid": "conv_centroid.cu",
               "fwd_finalize": "fwd.cu", "bwd_pre": "bwd.cu", "bwd_dq": "bwd.cu", "fwd_index": "index.cu",
               "bwd_index": "index.cu", "conv_bwd": "conv_bwd.cu"}
 

@@ -1,0 +1,367 @@
+// Backward of the sparse attention on the tcgen05 tensor cores.
+//
+// "Optimizing Mixture of Block Attention", §"Progettazione del Kernel
+// FlashMoBA", "Tre Kernel Fusi" 3 (backward parallel over key blocks, scores
+// recomputed, partial dQ accumulated with atomic adds into a high-precision
+// buffer) and §"Efficienza Backward Pass".  With the selection fixed:
+// P = exp(S/sqrt(d) - LSE), dS = P (.) (dO V^T - D), dV_j += P^T dO,
+// dK_j += dS^T Q / sqrt(d), dQ += dS K_j / sqrt(d).
+//
+// One CTA per (global key block j, KV head) walks the block's bucket of
+// gathered (query, head) rows in tiles of 128; thread t owns tile row t,
+// which is TMEM lane t.  Per tile:
+//   1. Q and dO rows are gathered (cp.async, 128-byte swizzled K-major) into
+//      one of two stages; the next tile's gather runs under this tile's work.
+//   2. One thread issues S = Q K_j^T and dP = dO V_j^T (M = 128 rows,
+//      N = B keys, K = d) into tensor memory.
+//   3. Each thread reads its row of S and dP (tcgen05.ld), forms P and dS in
+//      fp32 and stores them as bf16 tiles in shared memory.
+//   4. One thread issues dV_j^T += dO^T P and dK_j^T += Q^T dS (M = d, N = B,
+//      K = 128 rows; the same Q / dO tiles read M-major) and dQ = dS K_j
+//      (M = 128, N = d, K = B; K_j read N-major).  dV_j^T and dK_j^T stay in
+//      tensor memory for the whole bucket.
+//   5. Each thread reads its dQ row, scales it into a padded staging row and
+//      hands it to the TMA engine as one 4d-byte bulk fp32 reduction into the
+//      dQ accumulator.
+// At the end dK_j and dV_j are written once (bf16).  Every mbarrier wait is
+// bounded; a timeout sets MOBA_STATUS_TIMEOUT and the CTA winds down.
+#include "common.cuh"
+#include "launch.h"
+#include "tc.cuh"
+
+namespace moba {
+namespace {
+
+constexpr int kRows = 128;  // gathered rows per tile (= TMEM lanes)
+constexpr int kThreads = 128;
+
+template <int D, int BLK>
+struct BwdTcLayout {
+  static constexpr int KB = D / 64;                         // 64-wide d chunks (128-byte rows)
+  static constexpr uint32_t KV_REGION = BLK * 128;          // one d chunk of K_j or V_j
+  static constexpr uint32_t QO_REGION = kRows * 128;        // one d chunk of a Q or dO tile
+  static constexpr uint32_t PROW = BLK * 2;                 // bytes per row of the P / dS tiles
+  static constexpr uint32_t P_BYTES = kRows * PROW;
+  static constexpr uint32_t P_ATOM = BLK == 32 ? 512 : 1024; // bytes per 8-row group of P / dS
+  static constexpr uint32_t P_LAYOUT = BLK == 32 ? tc::kLayoutSW64 : tc::kLayoutSW128;
+  static constexpr uint32_t DQ_STRIDE = 4 * D + 16;         // staging row: fp32 dQ + pad (bank spread)
+  static constexpr uint32_t STAGE_QO = 2 * KB * QO_REGION;  // Q + dO
+  static constexpr uint32_t STAGE = (STAGE_QO > kRows * DQ_STRIDE ? STAGE_QO : kRows * DQ_STRIDE + 1023) / 1024 * 1024;
+  static constexpr uint32_t K_OFF = 0;
+  static constexpr uint32_t V_OFF = K_OFF + KB * KV_REGION;
+  static constexpr uint32_t P_OFF = V_OFF + KB * KV_REGION;
+  static constexpr uint32_t DS_OFF = P_OFF + P_BYTES;
+  static constexpr uint32_t ST_OFF = DS_OFF + P_BYTES;
+  static constexpr uint32_t MB_OFF = ST_OFF + 2 * STAGE;
+  static constexpr uint32_t HOLD_OFF = MB_OFF + 16;
+  static constexpr uint32_t BYTES = HOLD_OFF + 16;
+  // Tensor memory columns: S, dP (B each), dQ (D), dV^T, dK^T (B each).
+  static constexpr uint32_t S_COL = 0, DP_COL = BLK, DQ_COL = 2 * BLK, DV_COL = 2 * BLK + D, DK_COL = 3 * BLK + D;
+  static constexpr uint32_t NCOLS = 4 * BLK + D;
+  static constexpr uint32_t TMEM_COLS = NCOLS <= 256 ? 256 : 512;
+  static_assert(NCOLS <= 512, "tensor memory");
+  static_assert(KV_REGION % 1024 == 0 && P_BYTES % 1024 == 0, "swizzle atoms stay aligned");
+};
+
+// Byte offset of the 16-byte chunk c of row r in a P / dS tile.
+template <int BLK>
+__device__ __forceinline__ uint32_t p_offset(int r, int c) {
+  if constexpr (BLK == 32) return tc::sw64_offset(r, c);
+  else return tc::sw128_offset(r, c);
+}
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(kThreads)
+bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
+              const bf16* __restrict__ dout, const float* __restrict__ lse, const float* __restrict__ dsum,
+              const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch, int nb_max,
+              int h_q, int h_kv, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
+              float* __restrict__ dqacc, bf16* __restrict__ dk, bf16* __restrict__ dv,
+              int32_t* __restrict__ status) {
+  using Ly = BwdTcLayout<D, BLK>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(sm);
+  const uint32_t mb_s = sbase + Ly::MB_OFF, mb_g = mb_s + 8;
+
+  const int gb = blockIdx.x;
+  const int kvh = blockIdx.y;
+  if (gb >= __ldg(blk_off + batch)) return;
+  const int bucket = kvh * nb_max + gb;
+  const int beg = __ldg(ptr + bucket), end = __ldg(ptr + bucket + 1);
+  const int s = upper_seq(blk_off, batch, gb);
+  const int t0 = __ldg(cu + s) + (gb - __ldg(blk_off + s)) * BLK;
+  const int t1 = min(t0 + BLK, __ldg(cu + s + 1));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t kv_stride = (size_t)h_kv * D;
+  const float scale = rsqrtf((float)D);
+  const float scale_log2 = kLog2e * scale;
+  const int ntiles = (end - beg + kRows - 1) / kRows;
+
+  // ---- K_j, V_j -> SW128 K-major (row = key, 64-wide d chunks as regions)
+  for (int i = tid; i < BLK * (D / 8); i += kThreads) {
+    const int r = i / (D / 8), c = i % (D / 8);
+    const bool ok = t0 + r < t1;
+    const size_t off = ok ? (size_t)(t0 + r) * kv_stride + (size_t)kvh * D + c * 8 : 0;
+    const uint32_t o = (c >> 3) * Ly::KV_REGION + tc::sw128_offset(r, c & 7);
+    cp_async16_zfill(sm + Ly::K_OFF + o, k + off, ok);
+    cp_async16_zfill(sm + Ly::V_OFF + o, v + off, ok);
+  }
+  cp_async_commit();
+
+  // Row metadata: thread t holds tile row t's (row id, token, lse * log2 e, D).
+  int rid = -1, tok = -1;
+  float lse2 = 0.f, dsm = 0.f;
+  auto load_meta = [&](int tile, int& r_, int& t_, float& l_, float& d_) {
+    const int e = beg + tile * kRows + tid;
+    r_ = -1;
+    t_ = -1;
+    l_ = 0.f;
+    d_ = 0.f;
+    if (tile < ntiles && e < end) {
+      r_ = __ldg(rows + e);
+      t_ = r_ / h_q;
+      l_ = __ldg(lse + r_) * kLog2e;
+      d_ = __ldg(dsum + r_);
+    }
+  };
+  // Gather this warp's 32 rows of a tile (row ids from the lanes' `r_`):
+  // D/8 lanes per row, so each instruction moves whole 128-byte lines.
+  auto gather = [&](int stage, int r_) {
+    constexpr int LPR = D / 8;          // lanes per row
+    constexpr int RPI = 32 / LPR;       // rows per instruction
+    unsigned char* qs = sm + Ly::ST_OFF + stage * Ly::STAGE;
+    unsigned char* os = qs + Ly::KB * Ly::QO_REGION;
+    const int c = lane % LPR;
+#pragma unroll
+    for (int it = 0; it < 32 / RPI; ++it) {
+      const int rl = it * RPI + lane / LPR;
+      const int row = __shfl_sync(0xffffffffu, r_, rl);
+      const int tr = warp * 32 + rl;
+      const bool ok = row >= 0;
+      const size_t off = ok ? (size_t)row * D + c * 8 : 0;  // [T, H_q, D]: row t*H_q + h
+      const uint32_t o = (c >> 3) * Ly::QO_REGION + tc::sw128_offset(tr, c & 7);
+      cp_async16_zfill(qs + o, q + off, ok);
+      cp_async16_zfill(os + o, dout + off, ok);
+    }
+  };
+
+  if (tid == 0) {
+    tc::mbar_init(mb_s, 1);
+    tc::mbar_init(mb_g, 1);
+    tc::mbar_init_fence();
+  }
+  if (warp == 0) tc::tmem_alloc(sbase + Ly::HOLD_OFF, Ly::TMEM_COLS);
+  load_meta(0, rid, tok, lse2, dsm);
+  if (ntiles > 0) gather(0, rid);
+  cp_async_commit();
+  int nrid, ntok;
+  float nlse2, ndsm;
+  load_meta(1, nrid, ntok, nlse2, ndsm);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+
+  constexpr uint32_t id_s = tc::idesc_bf16_f32_major(kRows, BLK, 0, 0);  // S, dP
+  constexpr uint32_t id_g = tc::idesc_bf16_f32_major(D, BLK, 1, 1);      // dV^T, dK^T
+  constexpr uint32_t id_q = tc::idesc_bf16_f32_major(kRows, D, 0, 1);    // dQ
+
+  bool ok = true;
+  int fail_it = 0;
+  for (int it = 0; it < ntiles; ++it) {
+    fail_it = it;
+    const int stage = it & 1;
+    const uint32_t qa = sbase + Ly::ST_OFF + stage * Ly::STAGE;
+    const uint32_t oa = qa + Ly::KB * Ly::QO_REGION;
+    // A. this tile's rows (and, the first time, K_j / V_j) have landed
+    cp_async_wait<0>();
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    // B. S = Q K_j^T, dP = dO V_j^T
+    if (tid == 0) {
+      tc::fence_after_sync();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t ko = (kk >> 2) * Ly::QO_REGION + (kk & 3) * 32;
+        const uint32_t kb = (kk >> 2) * Ly::KV_REGION + (kk & 3) * 32;
+        tc::mma_bf16_ss(tmem + Ly::S_COL, tc::smem_desc(qa + ko, 16, 1024, tc::kLayoutSW128),
+                        tc::smem_desc(sbase + Ly::K_OFF + kb, 16, 1024, tc::kLayoutSW128), id_s, kk > 0);
+        tc::mma_bf16_ss(tmem + Ly::DP_COL, tc::smem_desc(oa + ko, 16, 1024, tc::kLayoutSW128),
+                        tc::smem_desc(sbase + Ly::V_OFF + kb, 16, 1024, tc::kLayoutSW128), id_s, kk > 0);
+      }
+      tc::mma_commit(mb_s);
+    }
+    // C. P and dS rows
+    {
+      const bool got = tc::mbar_wait(mb_s, it & 1);
+      if (!__syncthreads_and(got)) {
+        ok = false;
+        break;
+      }
+    }
+    tc::fence_after_sync();
+#pragma unroll
+    for (int h = 0; h < BLK / 32; ++h) {
+      uint32_t sv[32], pv[32];
+      tc::tmem_ld32(tmem + lane_base + Ly::S_COL + h * 32, sv);
+      tc::tmem_ld32(tmem + lane_base + Ly::DP_COL + h * 32, pv);
+      tc::tmem_ld_wait();
+      uint32_t pp[16], dd[16];
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        float p2[2], d2[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int key_tok = t0 + h * 32 + c + u;
+          float p = 0.f;
+          if (key_tok <= tok && key_tok < t1) p = fast_exp2(__uint_as_float(sv[c + u]) * scale_log2 - lse2);
+          p2[u] = p;
+          d2[u] = p * (__uint_as_float(pv[c + u]) - dsm);
+        }
+        pp[c / 2] = pack_bf16(p2[0], p2[1]);
+        dd[c / 2] = pack_bf16(d2[0], d2[1]);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t o = p_offset<BLK>(tid, h * 4 + c);
+        *reinterpret_cast<uint4*>(sm + Ly::P_OFF + o) = make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
+        *reinterpret_cast<uint4*>(sm + Ly::DS_OFF + o) = make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
+      }
+    }
+    tc::fence_proxy_async();
+    bulk_wait_read_all();  // the previous tile's dQ staging (next stage) has been read
+    tc::fence_before_sync();
+    __syncthreads();
+    // D. dV^T += dO^T P, dK^T += Q^T dS, dQ = dS K_j; next tile's gather
+    if (tid == 0) {
+      tc::fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < kRows / 16; ++ks) {
+        // 16 rows = two 8-row groups of the Q / dO tiles and of P / dS
+        const uint32_t ro = ks * 2048;
+        const uint32_t po = ks * 2 * Ly::P_ATOM;
+        const uint64_t pdesc = tc::smem_desc(sbase + Ly::P_OFF + po, 16, Ly::P_ATOM, Ly::P_LAYOUT);
+        const uint64_t sdesc = tc::smem_desc(sbase + Ly::DS_OFF + po, 16, Ly::P_ATOM, Ly::P_LAYOUT);
+        tc::mma_bf16_ss(tmem + Ly::DV_COL, tc::smem_desc(oa + ro, Ly::QO_REGION, 1024, tc::kLayoutSW128), pdesc,
+                        id_g, (it > 0 || ks > 0) ? 1u : 0u);
+        tc::mma_bf16_ss(tmem + Ly::DK_COL, tc::smem_desc(qa + ro, Ly::QO_REGION, 1024, tc::kLayoutSW128), sdesc,
+                        id_g, (it > 0 || ks > 0) ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < BLK / 16; ++kk) {
+        // K steps of 16 keys: 32 bytes along a dS row; two 8-key groups of K_j
+        tc::mma_bf16_ss(tmem + Ly::DQ_COL, tc::smem_desc(sbase + Ly::DS_OFF + kk * 32, 16, Ly::P_ATOM, Ly::P_LAYOUT),
+                        tc::smem_desc(sbase + Ly::K_OFF + kk * 2048, Ly::KV_REGION, 1024, tc::kLayoutSW128), id_q,
+                        kk > 0);
+      }
+      tc::mma_commit(mb_g);
+    }
+    if (it + 1 < ntiles) gather(stage ^ 1, nrid);
+    cp_async_commit();
+    // E. dQ rows -> staging -> bulk fp32 reduction
+    {
+      const bool got = tc::mbar_wait(mb_g, it & 1);
+      if (!__syncthreads_and(got)) {
+        ok = false;
+        break;
+      }
+    }
+    tc::fence_after_sync();
+    unsigned char* stg = sm + Ly::ST_OFF + stage * Ly::STAGE + (size_t)tid * Ly::DQ_STRIDE;
+#pragma unroll
+    for (int h = 0; h < D / 32; ++h) {
+      uint32_t qv[32];
+      tc::tmem_ld32(tmem + lane_base + Ly::DQ_COL + h * 32, qv);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<float4*>(stg + h * 128 + c * 16) =
+            make_float4(__uint_as_float(qv[4 * c]) * scale, __uint_as_float(qv[4 * c + 1]) * scale,
+                        __uint_as_float(qv[4 * c + 2]) * scale, __uint_as_float(qv[4 * c + 3]) * scale);
+    }
+    fence_proxy_async_smem();
+    if (rid >= 0) bulk_reduce_add_f32(dqacc + (size_t)rid * D, stg, 4 * D);
+    bulk_commit();
+    rid = nrid;
+    tok = ntok;
+    lse2 = nlse2;
+    dsm = ndsm;
+    load_meta(it + 2, nrid, ntok, nlse2, ndsm);
+  }
+  cp_async_wait<0>();
+  bulk_wait_all();
+  tc::fence_before_sync();
+  __syncthreads();
+  if (!ok) {
+    // A tensor-core completion never arrived: record it, give the MMAs in
+    // flight a bounded chance to drain, release TMEM, leave dK_j / dV_j alone.
+    if (tid == 0) set_status(status, kStatusTimeout);
+    tc::mbar_wait(mb_s, fail_it & 1, 100000000ull);
+    tc::mbar_wait(mb_g, fail_it & 1, 100000000ull);
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, Ly::TMEM_COLS);
+    return;
+  }
+  tc::fence_after_sync();
+  // dV_j^T, dK_j^T: accumulator row m (a d index) sits in lane m for M = 128,
+  // in lane (m % 16) + 32 (m / 16) for M = 64.
+  const int m = D == 128 ? tid : (lane < 16 ? warp * 16 + lane : -1);
+#pragma unroll
+  for (int h = 0; h < BLK / 32; ++h) {
+    uint32_t av[32], bv[32];
+    tc::tmem_ld32(tmem + lane_base + Ly::DV_COL + h * 32, av);
+    tc::tmem_ld32(tmem + lane_base + Ly::DK_COL + h * 32, bv);
+    tc::tmem_ld_wait();
+    if (m >= 0) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const int kt = t0 + h * 32 + c;
+        if (ntiles == 0) {
+          av[c] = 0u;
+          bv[c] = 0u;
+        }
+        if (kt < t1) {
+          const size_t o = (size_t)kt * kv_stride + (size_t)kvh * D + m;
+          dv[o] = __float2bfloat16_rn(__uint_as_float(av[c]));
+          dk[o] = __float2bfloat16_rn(__uint_as_float(bv[c]) * scale);
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, Ly::TMEM_COLS);
+}
+
+}  // namespace
+
+bool bwd_tc_supported(int d, int block_size) {
+  return (d == 64 && block_size == 32) || (d == 128 && (block_size == 32 || block_size == 64));
+}
+
+cudaError_t launch_bwd_tc(const bf16* q, const bf16* k, const bf16* v, const bf16* dout, const float* lse,
+                          const float* dsum, const SeqPlan& p, const int32_t* ptr, const int32_t* rows, int h_q,
+                          int h_kv, int d, int block_size, float* dqacc, bf16* dk, bf16* dv, int32_t* status,
+                          cudaStream_t st) {
+#define MOBA_BWD_TC(DD, BB)                                                                                  \
+  do {                                                                                                       \
+    const size_t smem = BwdTcLayout<DD, BB>::BYTES + 1024;                                                   \
+    auto kern = bwd_tc_kernel<DD, BB>;                                                                       \
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);     \
+    if (e != cudaSuccess) return e;                                                                          \
+    if (p.nb_max == 0) return cudaSuccess;                                                                   \
+    kern<<<dim3(p.nb_max, h_kv), kThreads, smem, st>>>(q, k, v, dout, lse, dsum, p.cu, p.blk_off, p.batch,   \
+                                                       p.nb_max, h_q, h_kv, ptr, rows, dqacc, dk, dv, status); \
+    return cudaGetLastError();                                                                               \
+  } while (0)
+  if (d == 64 && block_size == 32) MOBA_BWD_TC(64, 32);
+  if (d == 128 && block_size == 32) MOBA_BWD_TC(128, 32);
+  if (d == 128 && block_size == 64) MOBA_BWD_TC(128, 64);
+#undef MOBA_BWD_TC
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moba

@@ -68,6 +68,14 @@ cudaError_t launch_bwd_attn(const bf16* q, const bf16* k, const bf16* v, const b
                             const int32_t* rows, int h_q, int h_kv, int d, int block_size,
                             float* dqacc, bf16* dk, bf16* dv, cudaStream_t st);
 
+// tcgen05 backward attention (dK, dV written; dQ added into dqacc); the
+// shapes it covers (d, B) = (64, 32), (128, 32), (128, 64).
+bool bwd_tc_supported(int d, int block_size);
+cudaError_t launch_bwd_tc(const bf16* q, const bf16* k, const bf16* v, const bf16* dout, const float* lse,
+                          const float* dsum, const SeqPlan& p, const int32_t* ptr, const int32_t* rows, int h_q,
+                          int h_kv, int d, int block_size, float* dqacc, bf16* dk, bf16* dv, int32_t* status,
+                          cudaStream_t st);
+
 cudaError_t launch_bwd_dq(const float* dqacc, int n, bf16* dq, cudaStream_t st);
 
 // dw_part: h_kv * nb_max * d * conv_width floats of per-block partial sums.

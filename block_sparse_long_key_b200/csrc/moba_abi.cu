@@ -322,10 +322,17 @@ int moba_backward(const void* q, const void* k, const void* v, const void* out, 
                                 b.dqacc, st));
   STAGE_END(MOBA_STAGE_BWD_PRE);
   STAGE_BEGIN(MOBA_STAGE_BWD_ATTN);
-  MOBA_TRY(moba::launch_bwd_attn(static_cast<const bf16*>(q), static_cast<const bf16*>(k),
+  if (moba::bwd_tc_supported(d, shape->block_size)) {
+    MOBA_TRY(moba::launch_bwd_tc(static_cast<const bf16*>(q), static_cast<const bf16*>(k),
                                  static_cast<const bf16*>(v), static_cast<const bf16*>(dout), lse, b.dsum, plan, ptr,
                                  rows, hq, hkv, d, shape->block_size, b.dqacc, static_cast<bf16*>(dk),
-                                 static_cast<bf16*>(dv), st));
+                                 static_cast<bf16*>(dv), b.plan.status, st));
+  } else {
+    MOBA_TRY(moba::launch_bwd_attn(static_cast<const bf16*>(q), static_cast<const bf16*>(k),
+                                   static_cast<const bf16*>(v), static_cast<const bf16*>(dout), lse, b.dsum, plan, ptr,
+                                   rows, hq, hkv, d, shape->block_size, b.dqacc, static_cast<bf16*>(dk),
+                                   static_cast<bf16*>(dv), st));
+  }
   STAGE_END(MOBA_STAGE_BWD_ATTN);
   STAGE_BEGIN(MOBA_STAGE_BWD_DQ);
   MOBA_TRY(moba::launch_bwd_dq(b.dqacc, T * hq * d, static_cast<bf16*>(dq), st));

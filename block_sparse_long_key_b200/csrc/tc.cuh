@@ -33,6 +33,37 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
   return d;
 }
 
+// Byte offset of the 16-byte chunk `c` (8 bf16) of row `r` in a SW64 region
+// whose rows are 64 bytes (32 bf16) wide: 8 rows per 512-byte atom, chunk c
+// stored at c ^ ((r / 2) % 4).
+__device__ __forceinline__ uint32_t sw64_offset(int r, int c) {
+  return (uint32_t)((r >> 3) * 512 + (r & 7) * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+}
+
+constexpr uint32_t kLayoutSW128 = 2;
+constexpr uint32_t kLayoutSW64 = 4;
+
+// General shared-memory matrix descriptor.  K-major swizzled operands use
+// `sbo` = byte distance between 8-row groups (the leading offset is unused);
+// MN-major ones use `lbo` = byte distance between swizzle-wide groups along
+// M/N and `sbo` = byte distance between 8-row groups along K.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t smem_addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)layout << 61;
+  return d;
+}
+
+// Instruction descriptor with the operand majorness: a_mn / b_mn = 1 when A
+// (M x K) / B (N x K) is stored M- / N-contiguous instead of K-contiguous.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // Instruction descriptor: kind::f16 with bf16 A and B, fp32 accumulator,
 // both operands K-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
