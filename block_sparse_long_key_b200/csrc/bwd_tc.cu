@@ -10,21 +10,24 @@
 // One CTA per (global key block j, KV head) walks the block's bucket of
 // gathered (query, head) rows in tiles of 128; thread t owns tile row t,
 // which is TMEM lane t.  Per tile:
-//   1. Q and dO rows are gathered (cp.async, 128-byte swizzled K-major) into
-//      one of two stages; the next tile's gather runs under this tile's work.
+//   1. Q and dO rows are gathered (cp.async, 128-byte swizzled K-major).
 //   2. One thread issues S = Q K_j^T and dP = dO V_j^T (M = 128 rows,
 //      N = B keys, K = d) into tensor memory.
 //   3. Each thread reads its row of S and dP (tcgen05.ld), forms P and dS in
 //      fp32 and stores them as bf16 tiles in shared memory.
 //   4. One thread issues dV_j^T += dO^T P and dK_j^T += Q^T dS (M = d, N = B,
 //      K = 128 rows; the same Q / dO tiles read M-major) and dQ = dS K_j
-//      (M = 128, N = d, K = B; K_j read N-major).  dV_j^T and dK_j^T stay in
-//      tensor memory for the whole bucket.
-//   5. Each thread reads its dQ row, scales it into a padded staging row and
-//      hands it to the TMA engine as one 4d-byte bulk fp32 reduction into the
-//      dQ accumulator.
-// At the end dK_j and dV_j are written once (bf16).  Every mbarrier wait is
-// bounded; a timeout sets MOBA_STATUS_TIMEOUT and the CTA winds down.
+//      (M = 128, N = d, K = B; K_j read N-major) into the columns S and dP
+//      used.  dV_j^T and dK_j^T stay in tensor memory for the whole bucket.
+//   5. Each thread reads its dQ row; the next tile's gather is issued (the
+//      Q / dO tiles are free once the MMAs completed) and the row is added
+//      to the fp32 dQ accumulator with 16-byte vector reductions, lane pairs
+//      covering whole 32-byte sectors.
+// The CTA is sequential; a small footprint (one gather stage, 128 TMEM
+// columns at d = 64) lets four CTAs share an SM so that their phases
+// overlap.  At the end dK_j and dV_j are written once (bf16).  Every
+// mbarrier wait is bounded; a timeout sets MOBA_STATUS_TIMEOUT and the CTA
+// winds down.
 #include "common.cuh"
 #include "launch.h"
 #include "tc.cuh"
@@ -37,30 +40,31 @@ constexpr int kThreads = 128;
 
 template <int D, int BLK>
 struct BwdTcLayout {
-  static constexpr int KB = D / 64;                         // 64-wide d chunks (128-byte rows)
-  static constexpr uint32_t KV_REGION = BLK * 128;          // one d chunk of K_j or V_j
-  static constexpr uint32_t QO_REGION = kRows * 128;        // one d chunk of a Q or dO tile
-  static constexpr uint32_t PROW = BLK * 2;                 // bytes per row of the P / dS tiles
+  static constexpr int KB = D / 64;                          // 64-wide d chunks (128-byte rows)
+  static constexpr uint32_t KV_REGION = BLK * 128;           // one d chunk of K_j or V_j
+  static constexpr uint32_t QO_REGION = kRows * 128;         // one d chunk of a Q or dO tile
+  static constexpr uint32_t PROW = BLK * 2;                  // bytes per row of the P / dS tiles
   static constexpr uint32_t P_BYTES = kRows * PROW;
-  static constexpr uint32_t P_ATOM = BLK == 32 ? 512 : 1024; // bytes per 8-row group of P / dS
+  static constexpr uint32_t P_ATOM = BLK == 32 ? 512 : 1024;  // bytes per 8-row group of P / dS
   static constexpr uint32_t P_LAYOUT = BLK == 32 ? tc::kLayoutSW64 : tc::kLayoutSW128;
-  static constexpr uint32_t DQ_STRIDE = 4 * D + 16;         // staging row: fp32 dQ + pad (bank spread)
-  static constexpr uint32_t STAGE_QO = 2 * KB * QO_REGION;  // Q + dO
-  static constexpr uint32_t STAGE = (STAGE_QO > kRows * DQ_STRIDE ? STAGE_QO : kRows * DQ_STRIDE + 1023) / 1024 * 1024;
   static constexpr uint32_t K_OFF = 0;
   static constexpr uint32_t V_OFF = K_OFF + KB * KV_REGION;
   static constexpr uint32_t P_OFF = V_OFF + KB * KV_REGION;
   static constexpr uint32_t DS_OFF = P_OFF + P_BYTES;
-  static constexpr uint32_t ST_OFF = DS_OFF + P_BYTES;
-  static constexpr uint32_t MB_OFF = ST_OFF + 2 * STAGE;
+  static constexpr uint32_t Q_OFF = DS_OFF + P_BYTES;
+  static constexpr uint32_t O_OFF = Q_OFF + KB * QO_REGION;
+  static constexpr uint32_t MB_OFF = O_OFF + KB * QO_REGION;
   static constexpr uint32_t HOLD_OFF = MB_OFF + 16;
   static constexpr uint32_t BYTES = HOLD_OFF + 16;
-  // Tensor memory columns: S, dP (B each), dQ (D), dV^T, dK^T (B each).
-  static constexpr uint32_t S_COL = 0, DP_COL = BLK, DQ_COL = 2 * BLK, DV_COL = 2 * BLK + D, DK_COL = 3 * BLK + D;
-  static constexpr uint32_t NCOLS = 4 * BLK + D;
-  static constexpr uint32_t TMEM_COLS = NCOLS <= 256 ? 256 : 512;
+  // Tensor memory columns: S and dP side by side, later overwritten by dQ
+  // (D columns); then dV^T and dK^T (B each).
+  static constexpr uint32_t S_COL = 0, DP_COL = BLK, DQ_COL = 0;
+  static constexpr uint32_t DV_COL = (2 * BLK > D ? 2 * BLK : D), DK_COL = DV_COL + BLK;
+  static constexpr uint32_t NCOLS = DK_COL + BLK;
+  static constexpr uint32_t TMEM_COLS = NCOLS <= 128 ? 128 : (NCOLS <= 256 ? 256 : 512);
   static_assert(NCOLS <= 512, "tensor memory");
-  static_assert(KV_REGION % 1024 == 0 && P_BYTES % 1024 == 0, "swizzle atoms stay aligned");
+  static_assert(KV_REGION % 1024 == 0 && P_BYTES % 1024 == 0 && QO_REGION % 1024 == 0,
+                "swizzle atoms stay aligned");
 };
 
 // Byte offset of the 16-byte chunk c of row r in a P / dS tile.
@@ -107,31 +111,12 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
     cp_async16_zfill(sm + Ly::K_OFF + o, k + off, ok);
     cp_async16_zfill(sm + Ly::V_OFF + o, v + off, ok);
   }
-  cp_async_commit();
 
-  // Row metadata: thread t holds tile row t's (row id, token, lse * log2 e, D).
-  int rid = -1, tok = -1;
-  float lse2 = 0.f, dsm = 0.f;
-  auto load_meta = [&](int tile, int& r_, int& t_, float& l_, float& d_) {
-    const int e = beg + tile * kRows + tid;
-    r_ = -1;
-    t_ = -1;
-    l_ = 0.f;
-    d_ = 0.f;
-    if (tile < ntiles && e < end) {
-      r_ = __ldg(rows + e);
-      t_ = r_ / h_q;
-      l_ = __ldg(lse + r_) * kLog2e;
-      d_ = __ldg(dsum + r_);
-    }
-  };
   // Gather this warp's 32 rows of a tile (row ids from the lanes' `r_`):
   // D/8 lanes per row, so each instruction moves whole 128-byte lines.
-  auto gather = [&](int stage, int r_) {
-    constexpr int LPR = D / 8;          // lanes per row
-    constexpr int RPI = 32 / LPR;       // rows per instruction
-    unsigned char* qs = sm + Ly::ST_OFF + stage * Ly::STAGE;
-    unsigned char* os = qs + Ly::KB * Ly::QO_REGION;
+  auto gather = [&](int r_) {
+    constexpr int LPR = D / 8;     // lanes per row
+    constexpr int RPI = 32 / LPR;  // rows per instruction
     const int c = lane % LPR;
 #pragma unroll
     for (int it = 0; it < 32 / RPI; ++it) {
@@ -141,9 +126,16 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
       const bool ok = row >= 0;
       const size_t off = ok ? (size_t)row * D + c * 8 : 0;  // [T, H_q, D]: row t*H_q + h
       const uint32_t o = (c >> 3) * Ly::QO_REGION + tc::sw128_offset(tr, c & 7);
-      cp_async16_zfill(qs + o, q + off, ok);
-      cp_async16_zfill(os + o, dout + off, ok);
+      cp_async16_zfill(sm + Ly::Q_OFF + o, q + off, ok);
+      cp_async16_zfill(sm + Ly::O_OFF + o, dout + off, ok);
     }
+  };
+  // Row metadata (thread t: tile row t): row id, LSE and D.  The next
+  // tile's row id is loaded at the top of a tile and its statistics after
+  // the scores, so no load is waited for on the critical path.
+  auto meta_rid = [&](int tile) -> int {
+    const int e = beg + tile * kRows + tid;
+    return (tile < ntiles && e < end) ? __ldg(rows + e) : -1;
   };
 
   if (tid == 0) {
@@ -152,29 +144,26 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
     tc::mbar_init_fence();
   }
   if (warp == 0) tc::tmem_alloc(sbase + Ly::HOLD_OFF, Ly::TMEM_COLS);
-  load_meta(0, rid, tok, lse2, dsm);
-  if (ntiles > 0) gather(0, rid);
+  int rid = meta_rid(0), nrid = -1;
+  if (ntiles > 0) gather(rid);
   cp_async_commit();
-  int nrid, ntok;
-  float nlse2, ndsm;
-  load_meta(1, nrid, ntok, nlse2, ndsm);
+  float lse_c = rid >= 0 ? __ldg(lse + rid) : 0.f, dsum_c = rid >= 0 ? __ldg(dsum + rid) : 0.f;
+  float lse_n = 0.f, dsum_n = 0.f;
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const uint32_t qa = sbase + Ly::Q_OFF, oa = sbase + Ly::O_OFF;
 
   constexpr uint32_t id_s = tc::idesc_bf16_f32_major(kRows, BLK, 0, 0);  // S, dP
   constexpr uint32_t id_g = tc::idesc_bf16_f32_major(D, BLK, 1, 1);      // dV^T, dK^T
   constexpr uint32_t id_q = tc::idesc_bf16_f32_major(kRows, D, 0, 1);    // dQ
 
   bool ok = true;
-  int fail_it = 0;
-  for (int it = 0; it < ntiles; ++it) {
-    fail_it = it;
-    const int stage = it & 1;
-    const uint32_t qa = sbase + Ly::ST_OFF + stage * Ly::STAGE;
-    const uint32_t oa = qa + Ly::KB * Ly::QO_REGION;
+  int it = 0;
+  for (; it < ntiles; ++it) {
+    nrid = meta_rid(it + 1);  // consumed by the gather at the end of this tile
     // A. this tile's rows (and, the first time, K_j / V_j) have landed
     cp_async_wait<0>();
     tc::fence_proxy_async();
@@ -195,47 +184,51 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
       tc::mma_commit(mb_s);
     }
     // C. P and dS rows
-    {
-      const bool got = tc::mbar_wait(mb_s, it & 1);
-      if (!__syncthreads_and(got)) {
-        ok = false;
-        break;
-      }
+    if (!__syncthreads_and(tc::mbar_wait(mb_s, it & 1))) {
+      ok = false;
+      break;
     }
     tc::fence_after_sync();
+    {
+      const int tok = rid >= 0 ? rid / h_q : -1;
+      const float lse2 = lse_c * kLog2e, dsm = dsum_c;
 #pragma unroll
-    for (int h = 0; h < BLK / 32; ++h) {
-      uint32_t sv[32], pv[32];
-      tc::tmem_ld32(tmem + lane_base + Ly::S_COL + h * 32, sv);
-      tc::tmem_ld32(tmem + lane_base + Ly::DP_COL + h * 32, pv);
-      tc::tmem_ld_wait();
-      uint32_t pp[16], dd[16];
+      for (int h = 0; h < BLK / 32; ++h) {
+        uint32_t sv[32], pv[32];
+        tc::tmem_ld32(tmem + lane_base + Ly::S_COL + h * 32, sv);
+        tc::tmem_ld32(tmem + lane_base + Ly::DP_COL + h * 32, pv);
+        tc::tmem_ld_wait();
+        uint32_t pp[16], dd[16];
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        float p2[2], d2[2];
+        for (int c = 0; c < 32; c += 2) {
+          float p2[2], d2[2];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int key_tok = t0 + h * 32 + c + u;
-          float p = 0.f;
-          if (key_tok <= tok && key_tok < t1) p = fast_exp2(__uint_as_float(sv[c + u]) * scale_log2 - lse2);
-          p2[u] = p;
-          d2[u] = p * (__uint_as_float(pv[c + u]) - dsm);
+          for (int u = 0; u < 2; ++u) {
+            const int key_tok = t0 + h * 32 + c + u;
+            float p = 0.f;
+            if (key_tok <= tok && key_tok < t1) p = fast_exp2(__uint_as_float(sv[c + u]) * scale_log2 - lse2);
+            p2[u] = p;
+            d2[u] = p * (__uint_as_float(pv[c + u]) - dsm);
+          }
+          pp[c / 2] = pack_bf16(p2[0], p2[1]);
+          dd[c / 2] = pack_bf16(d2[0], d2[1]);
         }
-        pp[c / 2] = pack_bf16(p2[0], p2[1]);
-        dd[c / 2] = pack_bf16(d2[0], d2[1]);
-      }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint32_t o = p_offset<BLK>(tid, h * 4 + c);
-        *reinterpret_cast<uint4*>(sm + Ly::P_OFF + o) = make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
-        *reinterpret_cast<uint4*>(sm + Ly::DS_OFF + o) = make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t o = p_offset<BLK>(tid, h * 4 + c);
+          *reinterpret_cast<uint4*>(sm + Ly::P_OFF + o) =
+              make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
+          *reinterpret_cast<uint4*>(sm + Ly::DS_OFF + o) =
+              make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
+        }
       }
     }
+    lse_n = nrid >= 0 ? __ldg(lse + nrid) : 0.f;
+    dsum_n = nrid >= 0 ? __ldg(dsum + nrid) : 0.f;
     tc::fence_proxy_async();
-    bulk_wait_read_all();  // the previous tile's dQ staging (next stage) has been read
     tc::fence_before_sync();
     __syncthreads();
-    // D. dV^T += dO^T P, dK^T += Q^T dS, dQ = dS K_j; next tile's gather
+    // D. dV^T += dO^T P, dK^T += Q^T dS, dQ = dS K_j
     if (tid == 0) {
       tc::fence_after_sync();
 #pragma unroll
@@ -243,12 +236,11 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
         // 16 rows = two 8-row groups of the Q / dO tiles and of P / dS
         const uint32_t ro = ks * 2048;
         const uint32_t po = ks * 2 * Ly::P_ATOM;
-        const uint64_t pdesc = tc::smem_desc(sbase + Ly::P_OFF + po, 16, Ly::P_ATOM, Ly::P_LAYOUT);
-        const uint64_t sdesc = tc::smem_desc(sbase + Ly::DS_OFF + po, 16, Ly::P_ATOM, Ly::P_LAYOUT);
-        tc::mma_bf16_ss(tmem + Ly::DV_COL, tc::smem_desc(oa + ro, Ly::QO_REGION, 1024, tc::kLayoutSW128), pdesc,
-                        id_g, (it > 0 || ks > 0) ? 1u : 0u);
-        tc::mma_bf16_ss(tmem + Ly::DK_COL, tc::smem_desc(qa + ro, Ly::QO_REGION, 1024, tc::kLayoutSW128), sdesc,
-                        id_g, (it > 0 || ks > 0) ? 1u : 0u);
+        const uint32_t acc = (it > 0 || ks > 0) ? 1u : 0u;
+        tc::mma_bf16_ss(tmem + Ly::DV_COL, tc::smem_desc(oa + ro, Ly::QO_REGION, 1024, tc::kLayoutSW128),
+                        tc::smem_desc(sbase + Ly::P_OFF + po, 16, Ly::P_ATOM, Ly::P_LAYOUT), id_g, acc);
+        tc::mma_bf16_ss(tmem + Ly::DK_COL, tc::smem_desc(qa + ro, Ly::QO_REGION, 1024, tc::kLayoutSW128),
+                        tc::smem_desc(sbase + Ly::DS_OFF + po, 16, Ly::P_ATOM, Ly::P_LAYOUT), id_g, acc);
       }
 #pragma unroll
       for (int kk = 0; kk < BLK / 16; ++kk) {
@@ -259,40 +251,56 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
       }
       tc::mma_commit(mb_g);
     }
-    if (it + 1 < ntiles) gather(stage ^ 1, nrid);
-    cp_async_commit();
-    // E. dQ rows -> staging -> bulk fp32 reduction
-    {
-      const bool got = tc::mbar_wait(mb_g, it & 1);
-      if (!__syncthreads_and(got)) {
-        ok = false;
-        break;
-      }
+    // E. the tiles are free once the MMAs completed: start the next gather,
+    // then add this tile's dQ rows.
+    if (!__syncthreads_and(tc::mbar_wait(mb_g, it & 1))) {
+      ok = false;
+      break;
     }
     tc::fence_after_sync();
-    unsigned char* stg = sm + Ly::ST_OFF + stage * Ly::STAGE + (size_t)tid * Ly::DQ_STRIDE;
+    if (it + 1 < ntiles) gather(nrid);
+    cp_async_commit();
+    const int prow = __shfl_xor_sync(0xffffffffu, rid, 1);  // the lane pair's other row
+    const bool even = (lane & 1) == 0;
 #pragma unroll
     for (int h = 0; h < D / 32; ++h) {
       uint32_t qv[32];
       tc::tmem_ld32(tmem + lane_base + Ly::DQ_COL + h * 32, qv);
       tc::tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<float4*>(stg + h * 128 + c * 16) =
-            make_float4(__uint_as_float(qv[4 * c]) * scale, __uint_as_float(qv[4 * c + 1]) * scale,
-                        __uint_as_float(qv[4 * c + 2]) * scale, __uint_as_float(qv[4 * c + 3]) * scale);
+      for (int j = 0; j < 4; ++j) {
+        // Even lane: own row cols 8j..8j+3, partner row cols 8j..8j+3.
+        // Odd lane: partner row cols 8j+4..8j+7, own row cols 8j+4..8j+7.
+        float send[4], mine[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float lo = __uint_as_float(qv[8 * j + u]) * scale, hi = __uint_as_float(qv[8 * j + 4 + u]) * scale;
+          send[u] = even ? hi : lo;
+          mine[u] = even ? lo : hi;
+        }
+        float got[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) got[u] = __shfl_xor_sync(0xffffffffu, send[u], 1);
+        const int col = h * 32 + 8 * j + (even ? 0 : 4);
+        // first: the even lane's row; second: the odd lane's row
+        const int r1 = even ? rid : prow, r2 = even ? prow : rid;
+        float v1[4], v2[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          v1[u] = even ? mine[u] : got[u];
+          v2[u] = even ? got[u] : mine[u];
+        }
+        if (r1 >= 0) red_add_v4(dqacc + (size_t)r1 * D + col, v1[0], v1[1], v1[2], v1[3]);
+        if (r2 >= 0) red_add_v4(dqacc + (size_t)r2 * D + col, v2[0], v2[1], v2[2], v2[3]);
+      }
     }
-    fence_proxy_async_smem();
-    if (rid >= 0) bulk_reduce_add_f32(dqacc + (size_t)rid * D, stg, 4 * D);
-    bulk_commit();
+    tc::fence_before_sync();
     rid = nrid;
-    tok = ntok;
-    lse2 = nlse2;
-    dsm = ndsm;
-    load_meta(it + 2, nrid, ntok, nlse2, ndsm);
+    lse_c = lse_n;
+    dsum_c = dsum_n;
   }
+  const int fail_it = it;
   cp_async_wait<0>();
-  bulk_wait_all();
   tc::fence_before_sync();
   __syncthreads();
   if (!ok) {
@@ -319,14 +327,12 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         const int kt = t0 + h * 32 + c;
-        if (ntiles == 0) {
-          av[c] = 0u;
-          bv[c] = 0u;
-        }
+        const float a = ntiles > 0 ? __uint_as_float(av[c]) : 0.f;
+        const float b = ntiles > 0 ? __uint_as_float(bv[c]) * scale : 0.f;
         if (kt < t1) {
           const size_t o = (size_t)kt * kv_stride + (size_t)kvh * D + m;
-          dv[o] = __float2bfloat16_rn(__uint_as_float(av[c]));
-          dk[o] = __float2bfloat16_rn(__uint_as_float(bv[c]) * scale);
+          dv[o] = __float2bfloat16_rn(a);
+          dk[o] = __float2bfloat16_rn(b);
         }
       }
     }
