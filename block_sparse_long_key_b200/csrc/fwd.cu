@@ -17,7 +17,7 @@
 // softmax is taken against a fixed reference M_i (computed by the router as
 // a lower bound of the query's largest logit), so the contributions of its k
 // blocks are plain sums, exp(z - M_i) v and exp(z - M_i), added with fp32
-// reductions into an accumulator row [O | l | pad] that stays L2-resident
+// reductions into an accumulator row [O | l | pad] (32-byte aligned) that stays L2-resident
 // while a head is processed (CTAs run block-major within one head).  fp32 keeps the
 // full relative precision whatever the offset z - M_i, so M_i only has to be
 // within ~60 of the true maximum; a row whose logits exceed M_i by more than
@@ -62,7 +62,7 @@ fwd_attn_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
                 int h_q, int h_kv, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
                 const float* __restrict__ mref, float* __restrict__ oacc, int32_t* __restrict__ flag) {
   constexpr int KC = BLK < 64 ? BLK : 64;  // keys per register chunk
-  constexpr int OS = D + 4;                // accumulator row: O (D), l, 3 pad
+  constexpr int OS = oacc_stride(D);       // accumulator row: O (D), l, padding
   constexpr unsigned FULL = 0xffffffffu;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   FwdSmem<D, BLK>& sm = *reinterpret_cast<FwdSmem<D, BLK>*>(smem_raw);
@@ -251,12 +251,12 @@ fwd_attn_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
 }
 
 // O = acc / l (bf16), LSE = M + log l; flagged rows are queued instead.
-// Accumulator rows are D + 4 floats: O, then l, then padding.
+// Accumulator rows are oacc_stride(D) floats: O, then l, then padding.
 __global__ void __launch_bounds__(256)
 fwd_finalize_kernel(const float* __restrict__ oacc, const float* __restrict__ mref,
                     const int32_t* __restrict__ flag, long long nchunks, int d8, bf16* __restrict__ out,
                     float* __restrict__ lse, int32_t* __restrict__ flag_list) {
-  const int os = d8 * 8 + 4;
+  const int os = oacc_stride(d8 * 8);
   for (long long i = blockIdx.x * 256LL + threadIdx.x; i < nchunks; i += (long long)gridDim.x * 256) {
     const long long row = i / d8;
     const int c = (int)(i % d8);

@@ -1,0 +1,305 @@
+// Forward sparse attention on the tcgen05 tensor cores.
+//
+// "Optimizing Mixture of Block Attention", §"Definizione del Compito"
+// (O = softmax(QK^T/sqrt(d)) V over the selected blocks only) and
+// §"Progettazione del Kernel FlashMoBA", "Tre Kernel Fusi" 2 (gather the
+// queries that chose a key block into dense tiles, dense GEMMs against the
+// block, scatter the results).
+//
+// One CTA per (global key block j, KV head) walks the block's bucket in
+// tiles of 128 gathered rows; thread t owns tile row t = TMEM lane t.
+//   1. Q rows are gathered (cp.async, 128-byte swizzled K-major).
+//   2. One thread issues S = Q K_j^T (M = 128, N = B, K = d).
+//   3. Each thread reads its S row, applies the causal cut of the own block
+//      and p = exp(z - M_i) against the row's fixed reference M_i (from the
+//      router), sums l, checks the overflow bound and stores P as bf16.
+//      The next tile's gather starts here: the Q tile is free once S is.
+//   4. One thread issues O = P V_j (M = 128, N = d, K = B; V_j read
+//      N-major) into the columns S used.
+//   5. Each thread reads its O row and adds it, and l, to the query's fp32
+//      accumulator row [O | l | pad] with 16-byte vector reductions (lane
+//      pairs cover whole 32-byte sectors).
+// The merge of a query's k blocks is therefore a plain sum; finalize divides
+// by l.  A CTA needs ~33 KB of shared memory and 64 TMEM columns at d = 64,
+// so several share an SM and overlap their phases.  Every mbarrier wait is
+// bounded; a timeout sets MOBA_STATUS_TIMEOUT and the CTA winds down.
+#include "common.cuh"
+#include "launch.h"
+#include "tc.cuh"
+
+namespace moba {
+namespace {
+
+constexpr int kRows = 128;  // gathered rows per tile (= TMEM lanes)
+constexpr int kThreads = 128;
+constexpr float kOverflowLog2 = 90.f;  // ~62 in natural-log units
+
+template <int D, int BLK>
+struct FwdTcLayout {
+  static constexpr int KB = D / 64;                          // 64-wide d chunks (128-byte rows)
+  static constexpr uint32_t KV_REGION = BLK * 128;           // one d chunk of K_j or V_j
+  static constexpr uint32_t Q_REGION = kRows * 128;          // one d chunk of the Q tile
+  static constexpr uint32_t PROW = BLK * 2;                  // bytes per P row
+  static constexpr uint32_t P_BYTES = kRows * PROW;
+  static constexpr uint32_t P_ATOM = BLK == 32 ? 512 : 1024;  // bytes per 8-row group of P
+  static constexpr uint32_t P_LAYOUT = BLK == 32 ? tc::kLayoutSW64 : tc::kLayoutSW128;
+  static constexpr uint32_t K_OFF = 0;
+  static constexpr uint32_t V_OFF = K_OFF + KB * KV_REGION;
+  static constexpr uint32_t Q_OFF = V_OFF + KB * KV_REGION;
+  static constexpr uint32_t P_OFF = Q_OFF + KB * Q_REGION;
+  static constexpr uint32_t MB_OFF = P_OFF + P_BYTES;
+  static constexpr uint32_t HOLD_OFF = MB_OFF + 16;
+  static constexpr uint32_t BYTES = HOLD_OFF + 16;
+  // Tensor memory: S (B columns), later overwritten by O (D columns).
+  static constexpr uint32_t NCOLS = BLK > D ? BLK : D;
+  static constexpr uint32_t TMEM_COLS = NCOLS <= 32 ? 32 : (NCOLS <= 64 ? 64 : (NCOLS <= 128 ? 128 : 256));
+  static_assert(KV_REGION % 1024 == 0 && P_BYTES % 1024 == 0 && Q_REGION % 1024 == 0, "swizzle atoms stay aligned");
+};
+
+template <int BLK>
+__device__ __forceinline__ uint32_t p_offset(int r, int c) {
+  if constexpr (BLK == 32) return tc::sw64_offset(r, c);
+  else return tc::sw128_offset(r, c);
+}
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(kThreads)
+fwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
+              const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch, int nb_max,
+              int h_q, int h_kv, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
+              const float* __restrict__ mref, float* __restrict__ oacc, int32_t* __restrict__ flag,
+              int32_t* __restrict__ status) {
+  using Ly = FwdTcLayout<D, BLK>;
+  constexpr int OS = oacc_stride(D);
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(sm);
+  const uint32_t mb_s = sbase + Ly::MB_OFF, mb_o = mb_s + 8;
+
+  const int gb = blockIdx.x;
+  const int kvh = blockIdx.y;
+  if (gb >= __ldg(blk_off + batch)) return;
+  const int bucket = kvh * nb_max + gb;
+  const int beg = __ldg(ptr + bucket), end = __ldg(ptr + bucket + 1);
+  if (beg >= end) return;
+  const int s = upper_seq(blk_off, batch, gb);
+  const int t0 = __ldg(cu + s) + (gb - __ldg(blk_off + s)) * BLK;
+  const int t1 = min(t0 + BLK, __ldg(cu + s + 1));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t kv_stride = (size_t)h_kv * D;
+  const float scale_log2 = kLog2e * rsqrtf((float)D);
+  const int ntiles = (end - beg + kRows - 1) / kRows;
+
+  // ---- K_j, V_j -> SW128 K-major (row = key, 64-wide d chunks as regions)
+  for (int i = tid; i < BLK * (D / 8); i += kThreads) {
+    const int r = i / (D / 8), c = i % (D / 8);
+    const bool ok = t0 + r < t1;
+    const size_t off = ok ? (size_t)(t0 + r) * kv_stride + (size_t)kvh * D + c * 8 : 0;
+    const uint32_t o = (c >> 3) * Ly::KV_REGION + tc::sw128_offset(r, c & 7);
+    cp_async16_zfill(sm + Ly::K_OFF + o, k + off, ok);
+    cp_async16_zfill(sm + Ly::V_OFF + o, v + off, ok);
+  }
+  // Gather this warp's 32 rows of a tile: D/8 lanes per row (whole lines).
+  auto gather = [&](int r_) {
+    constexpr int LPR = D / 8;
+    constexpr int RPI = 32 / LPR;
+    const int c = lane % LPR;
+#pragma unroll
+    for (int it = 0; it < 32 / RPI; ++it) {
+      const int rl = it * RPI + lane / LPR;
+      const int row = __shfl_sync(0xffffffffu, r_, rl);
+      const bool ok = row >= 0;
+      const size_t off = ok ? (size_t)row * D + c * 8 : 0;  // q is [T, H_q, D]: row t*H_q + h
+      const uint32_t o = (c >> 3) * Ly::Q_REGION + tc::sw128_offset(warp * 32 + rl, c & 7);
+      cp_async16_zfill(sm + Ly::Q_OFF + o, q + off, ok);
+    }
+  };
+  auto meta_rid = [&](int tile) -> int {
+    const int e = beg + tile * kRows + tid;
+    return (tile < ntiles && e < end) ? __ldg(rows + e) : -1;
+  };
+
+  if (tid == 0) {
+    tc::mbar_init(mb_s, 1);
+    tc::mbar_init(mb_o, 1);
+    tc::mbar_init_fence();
+  }
+  if (warp == 0) tc::tmem_alloc(sbase + Ly::HOLD_OFF, Ly::TMEM_COLS);
+  int rid = meta_rid(0), nrid = -1;
+  gather(rid);
+  cp_async_commit();
+  float mr_c = rid >= 0 ? __ldg(mref + rid) * kLog2e : 0.f, mr_n = 0.f;
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const uint32_t qa = sbase + Ly::Q_OFF;
+  constexpr uint32_t id_s = tc::idesc_bf16_f32_major(kRows, BLK, 0, 0);  // S = Q K^T
+  constexpr uint32_t id_o = tc::idesc_bf16_f32_major(kRows, D, 0, 1);    // O = P V
+
+  bool ok = true;
+  int it = 0;
+  for (; it < ntiles; ++it) {
+    nrid = meta_rid(it + 1);
+    // A. this tile's rows (and, the first time, K_j / V_j) have landed
+    cp_async_wait<0>();
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    // B. S = Q K_j^T
+    if (tid == 0) {
+      tc::fence_after_sync();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t ko = (kk >> 2) * Ly::Q_REGION + (kk & 3) * 32;
+        const uint32_t kb = (kk >> 2) * Ly::KV_REGION + (kk & 3) * 32;
+        tc::mma_bf16_ss(tmem, tc::smem_desc(qa + ko, 16, 1024, tc::kLayoutSW128),
+                        tc::smem_desc(sbase + Ly::K_OFF + kb, 16, 1024, tc::kLayoutSW128), id_s, kk > 0);
+      }
+      tc::mma_commit(mb_s);
+    }
+    // C. P row; the Q tile is free: gather the next tile meanwhile
+    if (!__syncthreads_and(tc::mbar_wait(mb_s, it & 1))) {
+      ok = false;
+      break;
+    }
+    tc::fence_after_sync();
+    if (it + 1 < ntiles) gather(nrid);
+    cp_async_commit();
+    float l = 0.f, mx = -INFINITY;
+    {
+      const int tok = rid >= 0 ? rid / h_q : -1;
+#pragma unroll
+      for (int h = 0; h < BLK / 32; ++h) {
+        uint32_t sv[32];
+        tc::tmem_ld32(tmem + lane_base + h * 32, sv);
+        tc::tmem_ld_wait();
+        uint32_t pp[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float p2[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int key_tok = t0 + h * 32 + c + u;
+            float p = 0.f;
+            if (key_tok <= tok && key_tok < t1) {
+              const float x = __uint_as_float(sv[c + u]) * scale_log2;
+              p = fast_exp2(x - mr_c);
+              mx = fmaxf(mx, x);
+              l += p;
+            }
+            p2[u] = p;
+          }
+          pp[c / 2] = pack_bf16(p2[0], p2[1]);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(sm + Ly::P_OFF + p_offset<BLK>(tid, h * 4 + c)) =
+              make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
+      }
+    }
+    mr_n = nrid >= 0 ? __ldg(mref + nrid) * kLog2e : 0.f;
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    // D. O = P V_j into the score columns
+    if (tid == 0) {
+      tc::fence_after_sync();
+#pragma unroll
+      for (int kk = 0; kk < BLK / 16; ++kk)
+        tc::mma_bf16_ss(tmem, tc::smem_desc(sbase + Ly::P_OFF + kk * 32, 16, Ly::P_ATOM, Ly::P_LAYOUT),
+                        tc::smem_desc(sbase + Ly::V_OFF + kk * 2048, Ly::KV_REGION, 1024, tc::kLayoutSW128), id_o,
+                        kk > 0);
+      tc::mma_commit(mb_o);
+    }
+    // E. add the O row and l to the accumulator
+    if (!__syncthreads_and(tc::mbar_wait(mb_o, it & 1))) {
+      ok = false;
+      break;
+    }
+    tc::fence_after_sync();
+    if (rid >= 0) {
+      atomicAdd(oacc + (size_t)rid * OS + D, l);
+      if (mx - mr_c > kOverflowLog2) flag[rid] = 1;
+    }
+    const int prow = __shfl_xor_sync(0xffffffffu, rid, 1);  // the lane pair's other row
+    const bool even = (lane & 1) == 0;
+    const int r1 = even ? rid : prow, r2 = even ? prow : rid;  // even lane's row, odd lane's row
+#pragma unroll
+    for (int h = 0; h < D / 32; ++h) {
+      uint32_t ov[32];
+      tc::tmem_ld32(tmem + lane_base + h * 32, ov);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        // Even lane: columns 8j..8j+3 of both rows; odd lane: 8j+4..8j+7.
+        float send[4], mine[4], got[4], v1[4], v2[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float lo = __uint_as_float(ov[8 * j + u]), hi = __uint_as_float(ov[8 * j + 4 + u]);
+          send[u] = even ? hi : lo;
+          mine[u] = even ? lo : hi;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) got[u] = __shfl_xor_sync(0xffffffffu, send[u], 1);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          v1[u] = even ? mine[u] : got[u];
+          v2[u] = even ? got[u] : mine[u];
+        }
+        const int col = h * 32 + 8 * j + (even ? 0 : 4);
+        if (r1 >= 0) red_add_v4(oacc + (size_t)r1 * OS + col, v1[0], v1[1], v1[2], v1[3]);
+        if (r2 >= 0) red_add_v4(oacc + (size_t)r2 * OS + col, v2[0], v2[1], v2[2], v2[3]);
+      }
+    }
+    tc::fence_before_sync();
+    rid = nrid;
+    mr_c = mr_n;
+  }
+  const int fail_it = it;
+  cp_async_wait<0>();
+  tc::fence_before_sync();
+  __syncthreads();
+  if (!ok) {
+    // A tensor-core completion never arrived: record it, give the MMAs in
+    // flight a bounded chance to drain, release TMEM.
+    if (tid == 0) set_status(status, kStatusTimeout);
+    tc::mbar_wait(mb_s, fail_it & 1, 100000000ull);
+    tc::mbar_wait(mb_o, fail_it & 1, 100000000ull);
+    __syncthreads();
+  }
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, Ly::TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+bool fwd_tc_supported(int d, int block_size) {
+  return (d == 64 && block_size == 32) || (d == 128 && (block_size == 32 || block_size == 64));
+}
+
+cudaError_t launch_fwd_tc(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p, const int32_t* ptr,
+                          const int32_t* rows, const float* mref, int h_q, int h_kv, int d, int block_size,
+                          float* oacc, int32_t* flag, int32_t* status, cudaStream_t st) {
+#define MOBA_FWD_TC(DD, BB)                                                                                   \
+  do {                                                                                                        \
+    const size_t smem = FwdTcLayout<DD, BB>::BYTES + 1024;                                                    \
+    auto kern = fwd_tc_kernel<DD, BB>;                                                                        \
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);      \
+    if (e != cudaSuccess) return e;                                                                           \
+    if (p.nb_max == 0) return cudaSuccess;                                                                    \
+    kern<<<dim3(p.nb_max, h_kv), kThreads, smem, st>>>(q, k, v, p.cu, p.blk_off, p.batch, p.nb_max, h_q,      \
+                                                       h_kv, ptr, rows, mref, oacc, flag, status);            \
+    return cudaGetLastError();                                                                                \
+  } while (0)
+  if (d == 64 && block_size == 32) MOBA_FWD_TC(64, 32);
+  if (d == 128 && block_size == 32) MOBA_FWD_TC(128, 32);
+  if (d == 128 && block_size == 64) MOBA_FWD_TC(128, 64);
+#undef MOBA_FWD_TC
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moba

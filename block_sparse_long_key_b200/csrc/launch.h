@@ -33,7 +33,9 @@ cudaError_t launch_conv_centroid(const bf16* k, const float* conv_w, int conv_wi
                                  bf16* cent_hi, bf16* cent_lo, cudaStream_t st);
 
 // Forward accumulator rows: O (d floats), l, 3 floats of padding.
-__host__ __device__ constexpr int oacc_stride(int d) { return d + 4; }
+// Forward accumulator row: O (d floats), l, padding to a 32-byte multiple so
+// that every row starts on an L2 sector.
+__host__ __device__ constexpr int oacc_stride(int d) { return d + 8; }
 
 cudaError_t launch_route(const bf16* q, const bf16* k, const bf16* cent_hi, const bf16* cent_lo,
                          const SeqPlan& p, int h_q, int h_kv, int d, int block_size, int topk,
@@ -51,6 +53,12 @@ cudaError_t launch_build_index(const int32_t* sel_idx, const SeqPlan& p, int h_q
 cudaError_t launch_fwd_attn(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p,
                             const int32_t* ptr, const int32_t* rows, const float* mref, int h_q,
                             int h_kv, int d, int block_size, float* oacc, int32_t* flag, cudaStream_t st);
+
+// tcgen05 forward attention for (d, B) = (64, 32), (128, 32), (128, 64).
+bool fwd_tc_supported(int d, int block_size);
+cudaError_t launch_fwd_tc(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p, const int32_t* ptr,
+                          const int32_t* rows, const float* mref, int h_q, int h_kv, int d, int block_size,
+                          float* oacc, int32_t* flag, int32_t* status, cudaStream_t st);
 
 cudaError_t launch_fwd_finalize(const float* oacc, const float* mref, const int32_t* flag, int nrows,
                                 int d, bf16* out, float* lse, int32_t* flag_list, cudaStream_t st);

@@ -257,7 +257,11 @@ int moba_forward(const void* q, const void* k, const void* v, const int32_t* cu_
                                     b.plan.status, st, b.chunk_cnt));
   STAGE_END(MOBA_STAGE_FWD_INDEX);
   STAGE_BEGIN(MOBA_STAGE_FWD_ATTN);
-  MOBA_TRY(moba::launch_fwd_attn(kq, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.flag, st));
+  if (moba::fwd_tc_supported(d, B))
+    MOBA_TRY(moba::launch_fwd_tc(kq, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.flag,
+                                 b.plan.status, st));
+  else
+    MOBA_TRY(moba::launch_fwd_attn(kq, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.flag, st));
   STAGE_END(MOBA_STAGE_FWD_ATTN);
   STAGE_BEGIN(MOBA_STAGE_FWD_FINALIZE);
   MOBA_TRY(moba::launch_fwd_finalize(b.oacc, b.mref, b.flag, T * hq, d, static_cast<bf16*>(out), lse,
