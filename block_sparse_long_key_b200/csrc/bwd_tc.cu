@@ -20,9 +20,10 @@
 //      (M = 128, N = d, K = B; K_j read N-major) into the columns S and dP
 //      used.  dV_j^T and dK_j^T stay in tensor memory for the whole bucket.
 //   5. Each thread reads its dQ row; the next tile's gather is issued (the
-//      Q / dO tiles are free once the MMAs completed) and the row is added
-//      to the fp32 dQ accumulator with 16-byte vector reductions, lane pairs
-//      covering whole 32-byte sectors.
+//      Q / dO tiles are free once the MMAs completed) and the rows are added
+//      to the fp32 dQ accumulator with 16-byte vector reductions, staged
+//      through the free P / dS tiles so that 8 lanes cover one 128-byte row
+//      piece per instruction.
 // The CTA is sequential; a small footprint (one gather stage, 128 TMEM
 // columns at d = 64) lets four CTAs share an SM so that their phases
 // overlap.  At the end dK_j and dV_j are written once (bf16).  Every
@@ -260,39 +261,29 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
     tc::fence_after_sync();
     if (it + 1 < ntiles) gather(nrid);
     cp_async_commit();
-    const int prow = __shfl_xor_sync(0xffffffffu, rid, 1);  // the lane pair's other row
-    const bool even = (lane & 1) == 0;
+    // dQ rows leave through the (now free) P / dS tiles: each warp stages
+    // 32-column halves of its 32 rows, then 8 lanes cover one 128-byte row
+    // piece per reduction instruction.
+    unsigned char* stg = sm + Ly::P_OFF + warp * 4096;
 #pragma unroll
     for (int h = 0; h < D / 32; ++h) {
       uint32_t qv[32];
       tc::tmem_ld32(tmem + lane_base + Ly::DQ_COL + h * 32, qv);
       tc::tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        // Even lane: own row cols 8j..8j+3, partner row cols 8j..8j+3.
-        // Odd lane: partner row cols 8j+4..8j+7, own row cols 8j+4..8j+7.
-        float send[4], mine[4];
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<float4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+            make_float4(__uint_as_float(qv[4 * c]) * scale, __uint_as_float(qv[4 * c + 1]) * scale,
+                        __uint_as_float(qv[4 * c + 2]) * scale, __uint_as_float(qv[4 * c + 3]) * scale);
+      __syncwarp();
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float lo = __uint_as_float(qv[8 * j + u]) * scale, hi = __uint_as_float(qv[8 * j + 4 + u]) * scale;
-          send[u] = even ? hi : lo;
-          mine[u] = even ? lo : hi;
-        }
-        float got[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) got[u] = __shfl_xor_sync(0xffffffffu, send[u], 1);
-        const int col = h * 32 + 8 * j + (even ? 0 : 4);
-        // first: the even lane's row; second: the odd lane's row
-        const int r1 = even ? rid : prow, r2 = even ? prow : rid;
-        float v1[4], v2[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          v1[u] = even ? mine[u] : got[u];
-          v2[u] = even ? got[u] : mine[u];
-        }
-        if (r1 >= 0) red_add_v4(dqacc + (size_t)r1 * D + col, v1[0], v1[1], v1[2], v1[3]);
-        if (r2 >= 0) red_add_v4(dqacc + (size_t)r2 * D + col, v2[0], v2[1], v2[2], v2[3]);
+      for (int i = 0; i < 8; ++i) {
+        const int rl = i * 4 + (lane >> 3), c = lane & 7;
+        const float4 val = *reinterpret_cast<const float4*>(stg + rl * 128 + ((c ^ (rl & 7)) << 4));
+        const int row = __shfl_sync(0xffffffffu, rid, rl);
+        if (row >= 0) red_add_v4(dqacc + (size_t)row * D + h * 32 + c * 4, val.x, val.y, val.z, val.w);
       }
+      __syncwarp();
     }
     tc::fence_before_sync();
     rid = nrid;

@@ -174,5 +174,26 @@ __device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity, uint64
   }
 }
 
+// Named barrier `id` over `count` threads (a multiple of 32); id 0 is the
+// CTA-wide barrier.
+__device__ __forceinline__ void named_bar(uint32_t id, uint32_t count) {
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Same, returning the AND of `pred` over the participating threads.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(count) : "memory");
+  return r != 0;
+}
+// One arrival on an mbarrier (release semantics at CTA scope).
+__device__ __forceinline__ void mbar_arrive(uint32_t addr) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
 }  // namespace tc
 }  // namespace moba
