@@ -22,6 +22,7 @@ N up to 256K tokens, block sizes 32-128, head dim 64/128):
 from __future__ import annotations
 
 import dataclasses
+import math
 from typing import Dict, List, Optional, Tuple
 
 import torch
@@ -158,3 +159,57 @@ def small(seqlens, h_q, h_kv, d, B, topk, conv_width=0, seed=0, name="small") ->
     """An ad-hoc workload for parity tests."""
     return Workload(name, tuple(int(x) for x in seqlens), h_q, h_kv, d, B, topk,
                     conv_width=conv_width, seed=seed)
+
+
+def snr_sequence(B: int, d: int, h: int, delta_mu_eff: float, m: int, seed: int, index: int,
+                 full: bool = True) -> dict:
+    """One sequence of the routing signal-to-noise harness (CPU, float64).
+
+    2B + 1 tokens, ``h`` heads (KV heads = query heads).  Keys are
+    g / sqrt(d) with g ~ N(0, I), so for a unit query q every key score
+    q.k ~ N(0, 1/d).  The query rows that are measured are the last token
+    (position 2B, the first token of block 2): a unit vector per head.  In
+    one of the two earlier blocks (``signal`` per head, uniform) ``m`` tokens
+    get + (delta_mu_eff / m) q_hat added, so that block's key sum is shifted
+    by delta_mu_eff along q.  Other query rows and V are plain N(0, 1).
+
+    Returns dict(q, k, v) as float64 arrays [2B+1, h, d] and ``signal`` [h]
+    (with ``full=False`` only k, the measured query rows ``q_last`` [h, d]
+    and ``signal``: enough to route).
+    """
+    g = _gen(seed, 1000 + index)
+    L = 2 * B + 1
+    k = torch.randn((L, h, d), generator=g, dtype=torch.float64) / math.sqrt(d)
+    qlast = torch.randn((h, d), generator=g, dtype=torch.float64)
+    qlast /= qlast.norm(dim=-1, keepdim=True)
+    signal = torch.randint(0, 2, (h,), generator=g)
+    for hh in range(h):
+        j = int(signal[hh])
+        toks = torch.randperm(B, generator=g)[:m] + j * B
+        k[toks, hh] += (delta_mu_eff / m) * qlast[hh]
+    if not full:
+        return dict(k=k.numpy(), q_last=qlast.numpy(), signal=signal.numpy())
+    q = torch.randn((L, h, d), generator=g, dtype=torch.float64)
+    q[L - 1] = qlast
+    v = torch.randn((L, h, d), generator=g, dtype=torch.float64)
+    return dict(q=q.numpy(), k=k.numpy(), v=v.numpy(), signal=signal.numpy())
+
+
+def snr_batch(B: int, d: int, h: int, n_seq: int, delta_mu_eff: float, m: int = 1, seed: int = 0) -> dict:
+    """``n_seq`` harness sequences packed varlen, as bf16 CPU tensors.
+
+    Keys: q, k, v [T, h, d] bf16, cu_seqlens, rows (token of each measured
+    query, per sequence), signal [n_seq, h].
+    """
+    qs, ks, vs, sig = [], [], [], []
+    for i in range(n_seq):
+        one = snr_sequence(B, d, h, delta_mu_eff, m, seed, i)
+        qs.append(torch.from_numpy(one["q"]))
+        ks.append(torch.from_numpy(one["k"]))
+        vs.append(torch.from_numpy(one["v"]))
+        sig.append(torch.from_numpy(one["signal"]))
+    seqlens = [2 * B + 1] * n_seq
+    cu = cu_seqlens_of(seqlens)
+    return dict(q=torch.cat(qs).float().to(torch.bfloat16), k=torch.cat(ks).float().to(torch.bfloat16),
+                v=torch.cat(vs).float().to(torch.bfloat16), cu_seqlens=cu,
+                rows=(cu[1:] - 1).tolist(), signal=torch.stack(sig).numpy())

@@ -64,6 +64,8 @@ __all__ = [
     "block_selected_by",
     "block_index",
     "key_conv_backward",
+    "router_snr",
+    "router_p_fail",
 ]
 
 # Largest finite bf16 value, (2 - 2^-7) * 2^127.
@@ -433,3 +435,24 @@ def key_conv_backward(k: np.ndarray, w: np.ndarray, cu_seqlens, dk_conv: np.ndar
                 dk[a:b][: L - l] += w[None, :, :, l] * g[l:]
             dw[:, :, l] += (g * shifted[l]).sum(axis=0)
     return dk, dw
+
+
+def router_snr(delta_mu_eff: float, d: int, block_size: int) -> float:
+    """Signal-to-noise ratio of the block router.
+
+    §"Architettura del Modello Statistico" 2: for the score difference
+    D = s_signal - s_noise of a signal block against one noise block,
+    E[D] = delta_mu_eff / B and Var(D) = 2 sigma^2 / B with sigma^2 = 1/d
+    for unit-scale vectors, so SNR = E[D] / sqrt(Var(D))
+    = delta_mu_eff * sqrt(d / (2 B)).
+    """
+    mean = delta_mu_eff / block_size
+    var = 2.0 / (d * block_size)
+    return mean / math.sqrt(var)
+
+
+def router_p_fail(snr: float) -> float:
+    """Probability that the noise block outscores the signal block, Phi(-SNR)
+    (§"Architettura del Modello Statistico" 2), with Phi the standard normal
+    CDF written through the complementary error function."""
+    return 0.5 * math.erfc(snr / math.sqrt(2.0))
