@@ -240,6 +240,37 @@ def oracle_sample(w: synth.Workload, seed: int, rows_per_step: int, steps: int, 
 
 # ----------------------------------------------------------------------------- our arm
 
+def dense_context(g, hq, hkv, moba_ms):
+    """Dense causal attention forward + backward through the library SDPA
+    (flash backend only; None if it is unavailable), timed like the step."""
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    T, _, d = g["q"].shape
+    q = g["q"].view(1, T, hq, d).transpose(1, 2).detach().requires_grad_(True)
+    k = g["k"].view(1, T, hkv, d).transpose(1, 2).repeat_interleave(hq // hkv, dim=1).detach().requires_grad_(True)
+    v = g["v"].view(1, T, hkv, d).transpose(1, 2).repeat_interleave(hq // hkv, dim=1).detach().requires_grad_(True)
+    do = g["dout"].view(1, T, hq, d).transpose(1, 2)
+    try:
+        with sdpa_kernel([SDPBackend.FLASH_ATTENTION]):
+            def one():
+                o = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)
+                o.backward(do)
+            for _ in range(2):
+                one()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n = 3
+            e0.record()
+            for _ in range(n):
+                one()
+            e1.record()
+            torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) / n
+    except RuntimeError as exc:
+        return {"impl": "torch SDPA flash backend", "unavailable": str(exc).splitlines()[0][:160]}
+    return {"impl": "torch SDPA flash backend (library), dense causal, same Q/K/V shapes, fwd+bwd",
+            "ms_per_step": round(t, 3), "dense_over_moba": round(t / moba_ms, 3)}
+
+
 def run_ours(args):
     from block_sparse_long_key_b200 import moba
 
@@ -279,6 +310,7 @@ def run_ours(args):
         if cw is not None:   # through the key conv: gradients of the original keys and of the weights
             moba.key_conv_backward(kd, cw, cud, B, dk, workspace=ws_b, dk=dk_in, dw=dw)
 
+    torch.cuda.reset_peak_memory_stats(dev)
     for _ in range(args.warmup):
         step(g["q"], g["k"], g["v"], g["dout"], g["cu_seqlens"], conv_w)
     torch.cuda.synchronize()
@@ -333,6 +365,15 @@ def run_ours(args):
                              ("4*B*d FLOP" if dom == "fwd_attn" else "10*B*d FLOP", pairs))
                 if dom in ("fwd_attn", "bwd_attn") else unit}
 
+    # Memory: every buffer of the step is a torch allocation, so the peak
+    # covers inputs, outputs and both workspaces.  For context, the dense
+    # router-score matrix a materialising implementation would hold.
+    nb = T // B + w.batch
+    memory = {"peak_allocated_bytes": int(torch.cuda.max_memory_allocated(dev)),
+              "fwd_workspace_bytes": int(moba.fwd_workspace_size(shape)),
+              "bwd_workspace_bytes": int(moba.bwd_workspace_size(shape)),
+              "router_scores_if_materialised_bytes": int(T) * hq * nb * 4}
+
     # End to end through the public API with host buffers.
     e2e = None
     if not args.no_e2e:
@@ -366,6 +407,12 @@ def run_ours(args):
         e2e = {"value": round(aggregate_value(flops, world, ems), 3), "unit": UNIT, "ms_per_step": round(ems, 3),
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": ne}
 
+    # Context only: dense causal attention (the library SDPA, flash backend)
+    # forward + backward on the same Q, K, V shapes.
+    dense = None
+    if rank == 0 and world == 1 and not args.no_dense:
+        dense = dense_context(g, hq, hkv, ms_max)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         vals, desc, cores = oracle_sample(w, seed, args.cpu_rows, 2, 1)
@@ -391,7 +438,8 @@ def run_ours(args):
             "pct_of_bf16_peak": round(100.0 * value / world / peak_t, 3),
             "peak_bf16_tflops": peak_t, "peak_source": peak_src,
             "stage_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
-            "pairs": pairs, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "pairs": pairs, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "memory": memory,
+            "dense_context": dense,
             "gpu_launches": (LAUNCHES_PER_STEP + (LAUNCHES_CONV_BWD if w.conv_width else 0)) * args.steps, "clocks": clocks.summary(), "device_status": status,
         }
         print(json.dumps(line), flush=True)
@@ -431,6 +479,7 @@ def main(argv=None):
                     help="override the KV head count (query heads scale with it); for small profiling runs")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention context timing")
     ap.add_argument("--cpu-rows", type=int, default=1500, help="oracle rows per CPU-baseline step")
     ap.add_argument("--ref-rows", type=int, default=400, help="oracle rows per --impl reference step")
     args = ap.parse_args(argv)

@@ -105,3 +105,17 @@ def test_stage_table_ignores_plans_without_a_stage(L):
     ok = ctypes.c_void_p(1 << 20)
     assert L.moba_key_conv_centroid(ok, None, 0, ok, ctypes.byref(s), None, ok, ok, 16, None) == moba.MOBA_EWORKSPACE
     assert L.moba_set_stage_events(None, 0) == moba.MOBA_OK
+
+
+def test_workspace_grows_linearly_with_sequence_length(L):
+    # Nothing of size N x n (router scores) or N x N is held.  The only
+    # term above linear is the index build's per-chunk block histogram
+    # (N/1024 x N/B ints per KV head, used only while N/B <= 16384), which
+    # stays a fraction of the linear pick buffer: the bytes per token grow
+    # by well under 10 % per doubling of N.
+    for hq, d, B, k in ((16, 64, 32, 32), (8, 128, 64, 16)):
+        sizes = [moba.fwd_workspace_size(_shape(total_tokens=n, h_q=hq, h_kv=hq, head_dim=d, block_size=B, topk=k))
+                 + moba.bwd_workspace_size(_shape(total_tokens=n, h_q=hq, h_kv=hq, head_dim=d, block_size=B, topk=k))
+                 for n in (1 << 16, 1 << 17, 1 << 18)]
+        per_tok = [sz / n for sz, n in zip(sizes, (1 << 16, 1 << 17, 1 << 18))]
+        assert per_tok[1] / per_tok[0] < 1.1 and per_tok[2] / per_tok[1] < 1.1
