@@ -8,7 +8,9 @@
 //
 // One CTA per (global key block j, KV head) walks the block's bucket in
 // tiles of 128 gathered rows; thread t owns tile row t = TMEM lane t.
-//   1. Q rows are gathered (cp.async, 128-byte swizzled K-major).
+//   1. Q rows are gathered by the TMA (tile::gather4, four rows per
+//      instruction, 128-byte swizzle) into a K-major tile; completion is
+//      counted in bytes on an mbarrier.
 //   2. One thread issues S = Q K_j^T (M = 128, N = B, K = d).
 //   3. Each thread reads its S row, applies the causal cut of the own block
 //      and p = exp(z - M_i) against the row's fixed reference M_i (from the
@@ -47,8 +49,8 @@ struct FwdTcLayout {
   static constexpr uint32_t V_OFF = K_OFF + KB * KV_REGION;
   static constexpr uint32_t Q_OFF = V_OFF + KB * KV_REGION;
   static constexpr uint32_t P_OFF = Q_OFF + KB * Q_REGION;
-  static constexpr uint32_t MB_OFF = P_OFF + P_BYTES;
-  static constexpr uint32_t HOLD_OFF = MB_OFF + 16;
+  static constexpr uint32_t MB_OFF = P_OFF + P_BYTES;    // mbS, mbO, mbQ
+  static constexpr uint32_t HOLD_OFF = MB_OFF + 24;
   static constexpr uint32_t BYTES = HOLD_OFF + 16;
   // Tensor memory: S (B columns), later overwritten by O (D columns).
   static constexpr uint32_t NCOLS = BLK > D ? BLK : D;
@@ -64,7 +66,7 @@ __device__ __forceinline__ uint32_t p_offset(int r, int c) {
 
 template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads)
-fwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
+fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__ k, const bf16* __restrict__ v,
               const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch, int nb_max,
               int h_q, int h_kv, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
               const float* __restrict__ mref, float* __restrict__ oacc, int32_t* __restrict__ flag,
@@ -74,7 +76,7 @@ fwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(sm);
-  const uint32_t mb_s = sbase + Ly::MB_OFF, mb_o = mb_s + 8;
+  const uint32_t mb_s = sbase + Ly::MB_OFF, mb_o = mb_s + 8, mb_q = mb_s + 16;
 
   const int gb = blockIdx.x;
   const int kvh = blockIdx.y;
@@ -99,19 +101,23 @@ fwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
     cp_async16_zfill(sm + Ly::K_OFF + o, k + off, ok);
     cp_async16_zfill(sm + Ly::V_OFF + o, v + off, ok);
   }
-  // Gather this warp's 32 rows of a tile: D/8 lanes per row (whole lines).
+  // Gather this warp's 32 rows of a tile with the TMA: lanes 0..7 each
+  // issue one gather4 per 64-wide d chunk for rows 4l .. 4l+3 (row ids from
+  // the lanes' `r_`; a missing row reads row 0, whose P is zero).
   auto gather = [&](int r_) {
-    constexpr int LPR = D / 8;
-    constexpr int RPI = 32 / LPR;
-    const int c = lane % LPR;
+    int ids[4];
 #pragma unroll
-    for (int it = 0; it < 32 / RPI; ++it) {
-      const int rl = it * RPI + lane / LPR;
-      const int row = __shfl_sync(0xffffffffu, r_, rl);
-      const bool ok = row >= 0;
-      const size_t off = ok ? (size_t)row * D + c * 8 : 0;  // q is [T, H_q, D]: row t*H_q + h
-      const uint32_t o = (c >> 3) * Ly::Q_REGION + tc::sw128_offset(warp * 32 + rl, c & 7);
-      cp_async16_zfill(sm + Ly::Q_OFF + o, q + off, ok);
+    for (int u = 0; u < 4; ++u) {
+      const int x = __shfl_sync(0xffffffffu, r_, 4 * (lane & 7) + u);
+      ids[u] = x >= 0 ? x : 0;
+    }
+    if (lane == 0) tc::mbar_arrive_expect_tx(mb_q, 32 * D * 2);
+    __syncwarp();
+    if (lane < 8) {
+#pragma unroll
+      for (int c = 0; c < Ly::KB; ++c)
+        tc::tma_gather4(sbase + Ly::Q_OFF + c * Ly::Q_REGION + (warp * 32 + 4 * lane) * 128, &tm_q, c * 64, ids[0],
+                        ids[1], ids[2], ids[3], mb_q);
     }
   };
   auto meta_rid = [&](int tile) -> int {
@@ -122,16 +128,17 @@ fwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
   if (tid == 0) {
     tc::mbar_init(mb_s, 1);
     tc::mbar_init(mb_o, 1);
+    tc::mbar_init(mb_q, kThreads / 32);
     tc::mbar_init_fence();
   }
   if (warp == 0) tc::tmem_alloc(sbase + Ly::HOLD_OFF, Ly::TMEM_COLS);
-  int rid = meta_rid(0), nrid = -1;
-  gather(rid);
   cp_async_commit();
+  int rid = meta_rid(0), nrid = -1;
   float mr_c = rid >= 0 ? __ldg(mref + rid) * kLog2e : 0.f, mr_n = 0.f;
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  gather(rid);
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
   const uint32_t qa = sbase + Ly::Q_OFF;
@@ -145,8 +152,12 @@ fwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
     // A. this tile's rows (and, the first time, K_j / V_j) have landed
     cp_async_wait<0>();
     tc::fence_proxy_async();
+    const bool landed = tc::mbar_wait(mb_q, it & 1);
     tc::fence_before_sync();
-    __syncthreads();
+    if (!__syncthreads_and(landed)) {
+      ok = false;
+      break;
+    }
     // B. S = Q K_j^T
     if (tid == 0) {
       tc::fence_after_sync();
@@ -166,7 +177,6 @@ fwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
     }
     tc::fence_after_sync();
     if (it + 1 < ntiles) gather(nrid);
-    cp_async_commit();
     float l = 0.f, mx = -INFINITY;
     {
       const int tok = rid >= 0 ? rid / h_q : -1;
@@ -267,6 +277,10 @@ fwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
     if (tid == 0) set_status(status, kStatusTimeout);
     tc::mbar_wait(mb_s, fail_it & 1, 100000000ull);
     tc::mbar_wait(mb_o, fail_it & 1, 100000000ull);
+    // A gather in flight (for this tile or the next) lands before exit: the
+    // wait on the phase that is not pending returns at once.
+    tc::mbar_wait(mb_q, fail_it & 1, 100000000ull);
+    tc::mbar_wait(mb_q, (fail_it + 1) & 1, 100000000ull);
     __syncthreads();
   }
   if (warp == 0) {
@@ -281,9 +295,9 @@ bool fwd_tc_supported(int d, int block_size) {
   return (d == 64 && block_size == 32) || (d == 128 && (block_size == 32 || block_size == 64));
 }
 
-cudaError_t launch_fwd_tc(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p, const int32_t* ptr,
-                          const int32_t* rows, const float* mref, int h_q, int h_kv, int d, int block_size,
-                          float* oacc, int32_t* flag, int32_t* status, cudaStream_t st) {
+cudaError_t launch_fwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const SeqPlan& p,
+                          const int32_t* ptr, const int32_t* rows, const float* mref, int h_q, int h_kv, int d,
+                          int block_size, float* oacc, int32_t* flag, int32_t* status, cudaStream_t st) {
 #define MOBA_FWD_TC(DD, BB)                                                                                   \
   do {                                                                                                        \
     const size_t smem = FwdTcLayout<DD, BB>::BYTES + 1024;                                                    \
@@ -291,7 +305,7 @@ cudaError_t launch_fwd_tc(const bf16* q, const bf16* k, const bf16* v, const Seq
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);      \
     if (e != cudaSuccess) return e;                                                                           \
     if (p.nb_max == 0) return cudaSuccess;                                                                    \
-    kern<<<dim3(p.nb_max, h_kv), kThreads, smem, st>>>(q, k, v, p.cu, p.blk_off, p.batch, p.nb_max, h_q,      \
+    kern<<<dim3(p.nb_max, h_kv), kThreads, smem, st>>>(tm_q, k, v, p.cu, p.blk_off, p.batch, p.nb_max, h_q,   \
                                                        h_kv, ptr, rows, mref, oacc, flag, status);            \
     return cudaGetLastError();                                                                                \
   } while (0)

@@ -4,6 +4,7 @@
 // include/moba.h and at each kernel.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -54,11 +55,17 @@ cudaError_t launch_fwd_attn(const bf16* q, const bf16* k, const bf16* v, const S
                             const int32_t* ptr, const int32_t* rows, const float* mref, int h_q,
                             int h_kv, int d, int block_size, float* oacc, int32_t* flag, cudaStream_t st);
 
-// tcgen05 forward attention for (d, B) = (64, 32), (128, 32), (128, 64).
+// Tensor map over a [nrows, d] bf16 row table (16-byte aligned base) for
+// the tile::gather4 row gathers: 64-element boxes one row high, 128-byte
+// swizzle.
+cudaError_t make_row_map(CUtensorMap* map, const void* base, unsigned long long nrows, int d);
+
+// tcgen05 forward attention for (d, B) = (64, 32), (128, 32), (128, 64);
+// `tm_q` is make_row_map over q as T*H_q rows.
 bool fwd_tc_supported(int d, int block_size);
-cudaError_t launch_fwd_tc(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p, const int32_t* ptr,
-                          const int32_t* rows, const float* mref, int h_q, int h_kv, int d, int block_size,
-                          float* oacc, int32_t* flag, int32_t* status, cudaStream_t st);
+cudaError_t launch_fwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const SeqPlan& p,
+                          const int32_t* ptr, const int32_t* rows, const float* mref, int h_q, int h_kv, int d,
+                          int block_size, float* oacc, int32_t* flag, int32_t* status, cudaStream_t st);
 
 cudaError_t launch_fwd_finalize(const float* oacc, const float* mref, const int32_t* flag, int nrows,
                                 int d, bf16* out, float* lse, int32_t* flag_list, cudaStream_t st);

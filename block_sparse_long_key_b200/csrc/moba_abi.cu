@@ -257,8 +257,9 @@ int moba_forward(const void* q, const void* k, const void* v, const int32_t* cu_
                                     b.plan.status, st, b.chunk_cnt));
   STAGE_END(MOBA_STAGE_FWD_INDEX);
   STAGE_BEGIN(MOBA_STAGE_FWD_ATTN);
-  if (moba::fwd_tc_supported(d, B))
-    MOBA_TRY(moba::launch_fwd_tc(kq, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.flag,
+  CUtensorMap tm_q;
+  if (moba::fwd_tc_supported(d, B) && moba::make_row_map(&tm_q, kq, (unsigned long long)T * hq, d) == cudaSuccess)
+    MOBA_TRY(moba::launch_fwd_tc(tm_q, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.flag,
                                  b.plan.status, st));
   else
     MOBA_TRY(moba::launch_fwd_attn(kq, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.flag, st));

@@ -190,6 +190,25 @@ __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool 
       : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(count) : "memory");
   return r != 0;
 }
+// Registers `bytes` of expected async transactions with one arrival.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t addr, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(bytes) : "memory");
+}
+
+// TMA row gather: rows r0..r3 of a 2-D tensor map (box: 64 elements x one
+// row, 128-byte swizzle), columns c0 .. c0+63, into 4 consecutive 128-byte
+// rows of shared memory at `dst` (128-byte aligned; the swizzle follows the
+// address bits, so a 1024-byte aligned tile gets the SW128 K-major layout).
+// Completion is counted in bytes on `mbar`.  No cluster multicast.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int c0, int r0, int r1, int r2, int r3,
+                                            uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(mbar)
+      : "memory");
+}
+
 // One arrival on an mbarrier (release semantics at CTA scope).
 __device__ __forceinline__ void mbar_arrive(uint32_t addr) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(addr) : "memory");
