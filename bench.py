@@ -48,10 +48,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel source file it was taken with: a changed source voids the figure.
 # Headline workload, one timed-step launch each (profiles/dram_traffic_n64k_h16_d64_b32_k32_kconv4.md).
 NCU_TRAFFIC = {
-    "fwd_route": {"bytes": 313.64e6 + 408.26e6, "sha": "6f9dfb1cc06a69b2"},
-    "fwd_attn": {"bytes": 1.02e9 + 668.09e6, "sha": "c12b24e4d39fbab2"},
-    "bwd_attn": {"bytes": 1.11e9 + 591.03e6, "sha": "860c3246646589a8"},
-    "conv_bwd": {"bytes": 269.38e6 + 131.24e6, "sha": "5f8d17997de2fc78"},
+    "fwd_route": {"bytes": 312.81e6 + 409.11e6, "sha": "e83003f4ed7f8895"},
+    "fwd_attn": {"bytes": 1.18e9 + 925.48e6, "sha": "89d8dbb64ffc1058"},
+    "bwd_attn": {"bytes": 1.09e9 + 577.66e6, "sha": "5c7885370225fbc4"},
+    "conv_bwd": {"bytes": 269.32e6 + 131.05e6, "sha": "5f8d17997de2fc78"},
 }
 
 
@@ -179,7 +179,7 @@ def stage_roofline(name, w, pairs, scored, peaks):
     return "hbm", 0.0, "byte"
 
 
-KERNEL_SRC = {"fwd_attn": "fwd.cu", "bwd_attn": "bwd_tc.cu", "fwd_route": "route.cu", "fwd_centroid": "conv_centroid.cu",
+KERNEL_SRC = {"fwd_attn": "fwd_tc.cu", "bwd_attn": "bwd_tc.cu", "fwd_route": "route.cu", "fwd_centroid": "conv_centroid.cu",
               "fwd_finalize": "fwd.cu", "bwd_pre": "bwd.cu", "bwd_dq": "bwd.cu", "fwd_index": "index.cu",
               "bwd_index": "index.cu", "conv_bwd": "conv_bwd.cu"}
 
