@@ -272,3 +272,32 @@ def test_key_conv_backward_matches_oracle(dev, case):
     assert np.all(err <= 2.0 ** -8 * np.abs(dk_r) + 1e-5 * rms), (err / (np.abs(dk_r) + rms)).max()
     # dW: fp32 sums over every token of a head.
     np.testing.assert_allclose(pu.to64(dw), dw_r, rtol=1e-3, atol=1e-4 * np.abs(dw_r).max())
+
+
+@pytest.mark.parametrize("d,B", [(64, 32), (128, 64)])
+def test_rows_far_above_the_reference_take_the_exact_path(dev, d, B):
+    # A key far above its block's mean along a later query (its logit ~190
+    # natural-log units above the centroid-based reference M_i) would
+    # overflow the fixed-reference sums; such rows are flagged and
+    # recomputed exactly (online softmax) and must still match the oracle.
+    w = synth.small((2048,), 2, 2, d, B, 8, seed=17)
+    x = synth.make_inputs(w)
+    i, h, j = 1500, 0, 5                      # query token, head, block of the planted key
+    qh = x["q"][i, h].float()
+    x["k"][j * B + 7, h] = (200.0 * qh / qh.norm()).to(torch.bfloat16)
+    g = _gpu(x, dev)
+    out, lse, sel, _ = moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], B, w.topk)
+    torch.cuda.synchronize()
+    ref = pu.oracle_forward(x, B, w.topk)
+    assert j in ref["sel"][i, h]               # the planted block is picked by that query
+    sel_g = sel.cpu().numpy()
+    bad = pu.selection_mismatch_rows(sel_g, ref["sel"], ref["gap"])   # near ties only
+    o_g, lse_g = pu.to64(out), pu.to64(lse)
+    assert np.isfinite(o_g).all() and np.isfinite(lse_g).all()
+    assert lse_g[i, h] > 100.0                 # the huge logit dominates
+    o_ref, lse_ref = ref["o"].copy(), ref["lse"].copy()
+    if bad:
+        o2, l2 = orc.attention(ref["q"], ref["k"], ref["v"], sel_g, ref["cu"], B, rows=bad)
+        for t, hh in bad:
+            o_ref[t, hh], lse_ref[t, hh] = o2[t, hh], l2[t, hh]
+    pu.check_o_lse(o_g, lse_g, o_ref, lse_ref, "overflow_d%d_B%d" % (d, B))
