@@ -10,7 +10,9 @@
 // One CTA per (global key block j, KV head) walks the block's bucket of
 // gathered (query, head) rows in tiles of 128; thread t owns tile row t,
 // which is TMEM lane t.  Per tile:
-//   1. Q and dO rows are gathered (cp.async, 128-byte swizzled K-major).
+//   1. Q and dO rows are gathered by the TMA (tile::gather4, four rows per
+//      instruction, 128-byte swizzle) into K-major tiles; completion is
+//      counted in bytes on an mbarrier.
 //   2. One thread issues S = Q K_j^T and dP = dO V_j^T (M = 128 rows,
 //      N = B keys, K = d) into tensor memory.
 //   3. Each thread reads its row of S and dP (tcgen05.ld), forms P and dS in
@@ -54,8 +56,8 @@ struct BwdTcLayout {
   static constexpr uint32_t DS_OFF = P_OFF + P_BYTES;
   static constexpr uint32_t Q_OFF = DS_OFF + P_BYTES;
   static constexpr uint32_t O_OFF = Q_OFF + KB * QO_REGION;
-  static constexpr uint32_t MB_OFF = O_OFF + KB * QO_REGION;
-  static constexpr uint32_t HOLD_OFF = MB_OFF + 16;
+  static constexpr uint32_t MB_OFF = O_OFF + KB * QO_REGION;  // mbS, mbG, mbQ
+  static constexpr uint32_t HOLD_OFF = MB_OFF + 24;
   static constexpr uint32_t BYTES = HOLD_OFF + 16;
   // Tensor memory columns: S and dP side by side, later overwritten by dQ
   // (D columns); then dV^T and dK^T (B each).
@@ -77,8 +79,8 @@ __device__ __forceinline__ uint32_t p_offset(int r, int c) {
 
 template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads)
-bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
-              const bf16* __restrict__ dout, const float* __restrict__ lse, const float* __restrict__ dsum,
+bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__ k, const bf16* __restrict__ v,
+              const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ lse, const float* __restrict__ dsum,
               const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch, int nb_max,
               int h_q, int h_kv, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
               float* __restrict__ dqacc, bf16* __restrict__ dk, bf16* __restrict__ dv,
@@ -87,7 +89,7 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(sm);
-  const uint32_t mb_s = sbase + Ly::MB_OFF, mb_g = mb_s + 8;
+  const uint32_t mb_s = sbase + Ly::MB_OFF, mb_g = mb_s + 8, mb_q = mb_s + 16;
 
   const int gb = blockIdx.x;
   const int kvh = blockIdx.y;
@@ -113,22 +115,28 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
     cp_async16_zfill(sm + Ly::V_OFF + o, v + off, ok);
   }
 
-  // Gather this warp's 32 rows of a tile (row ids from the lanes' `r_`):
-  // D/8 lanes per row, so each instruction moves whole 128-byte lines.
+  // Gather this warp's 32 rows of a tile with the TMA: lanes 0..7 each
+  // issue one gather4 per 64-wide d chunk and tensor for rows 4l .. 4l+3
+  // (row ids from the lanes' `r_`; a missing row reads row 0, whose P and dS
+  // are zero).
   auto gather = [&](int r_) {
-    constexpr int LPR = D / 8;     // lanes per row
-    constexpr int RPI = 32 / LPR;  // rows per instruction
-    const int c = lane % LPR;
+    int ids[4];
 #pragma unroll
-    for (int it = 0; it < 32 / RPI; ++it) {
-      const int rl = it * RPI + lane / LPR;
-      const int row = __shfl_sync(0xffffffffu, r_, rl);
-      const int tr = warp * 32 + rl;
-      const bool ok = row >= 0;
-      const size_t off = ok ? (size_t)row * D + c * 8 : 0;  // [T, H_q, D]: row t*H_q + h
-      const uint32_t o = (c >> 3) * Ly::QO_REGION + tc::sw128_offset(tr, c & 7);
-      cp_async16_zfill(sm + Ly::Q_OFF + o, q + off, ok);
-      cp_async16_zfill(sm + Ly::O_OFF + o, dout + off, ok);
+    for (int u = 0; u < 4; ++u) {
+      const int x = __shfl_sync(0xffffffffu, r_, 4 * (lane & 7) + u);
+      ids[u] = x >= 0 ? x : 0;
+    }
+    if (lane == 0) tc::mbar_arrive_expect_tx(mb_q, 2 * 32 * D * 2);
+    __syncwarp();
+    if (lane < 8) {
+      const uint32_t o = (warp * 32 + 4 * lane) * 128;
+#pragma unroll
+      for (int c = 0; c < Ly::KB; ++c) {
+        tc::tma_gather4(sbase + Ly::Q_OFF + c * Ly::QO_REGION + o, &tm_q, c * 64, ids[0], ids[1], ids[2], ids[3],
+                        mb_q);
+        tc::tma_gather4(sbase + Ly::O_OFF + c * Ly::QO_REGION + o, &tm_do, c * 64, ids[0], ids[1], ids[2], ids[3],
+                        mb_q);
+      }
     }
   };
   // Row metadata (thread t: tile row t): row id, LSE and D.  The next
@@ -142,17 +150,18 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
   if (tid == 0) {
     tc::mbar_init(mb_s, 1);
     tc::mbar_init(mb_g, 1);
+    tc::mbar_init(mb_q, kThreads / 32);
     tc::mbar_init_fence();
   }
   if (warp == 0) tc::tmem_alloc(sbase + Ly::HOLD_OFF, Ly::TMEM_COLS);
-  int rid = meta_rid(0), nrid = -1;
-  if (ntiles > 0) gather(rid);
   cp_async_commit();
+  int rid = meta_rid(0), nrid = -1;
   float lse_c = rid >= 0 ? __ldg(lse + rid) : 0.f, dsum_c = rid >= 0 ? __ldg(dsum + rid) : 0.f;
   float lse_n = 0.f, dsum_n = 0.f;
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  if (ntiles > 0) gather(rid);
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
   const uint32_t qa = sbase + Ly::Q_OFF, oa = sbase + Ly::O_OFF;
@@ -168,8 +177,12 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
     // A. this tile's rows (and, the first time, K_j / V_j) have landed
     cp_async_wait<0>();
     tc::fence_proxy_async();
+    const bool landed = tc::mbar_wait(mb_q, it & 1);
     tc::fence_before_sync();
-    __syncthreads();
+    if (!__syncthreads_and(landed)) {
+      ok = false;
+      break;
+    }
     // B. S = Q K_j^T, dP = dO V_j^T
     if (tid == 0) {
       tc::fence_after_sync();
@@ -260,7 +273,6 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
     }
     tc::fence_after_sync();
     if (it + 1 < ntiles) gather(nrid);
-    cp_async_commit();
     // dQ rows leave through the (now free) P / dS tiles: each warp stages
     // 32-column halves of its 32 rows, then 8 lanes cover one 128-byte row
     // piece per reduction instruction.
@@ -300,6 +312,9 @@ bwd_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16
     if (tid == 0) set_status(status, kStatusTimeout);
     tc::mbar_wait(mb_s, fail_it & 1, 100000000ull);
     tc::mbar_wait(mb_g, fail_it & 1, 100000000ull);
+    // a gather in flight (this tile's or the next) lands before exit
+    tc::mbar_wait(mb_q, fail_it & 1, 100000000ull);
+    tc::mbar_wait(mb_q, (fail_it + 1) & 1, 100000000ull);
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, Ly::TMEM_COLS);
     return;
@@ -339,10 +354,10 @@ bool bwd_tc_supported(int d, int block_size) {
   return (d == 64 && block_size == 32) || (d == 128 && (block_size == 32 || block_size == 64));
 }
 
-cudaError_t launch_bwd_tc(const bf16* q, const bf16* k, const bf16* v, const bf16* dout, const float* lse,
-                          const float* dsum, const SeqPlan& p, const int32_t* ptr, const int32_t* rows, int h_q,
-                          int h_kv, int d, int block_size, float* dqacc, bf16* dk, bf16* dv, int32_t* status,
-                          cudaStream_t st) {
+cudaError_t launch_bwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const CUtensorMap& tm_do,
+                          const float* lse, const float* dsum, const SeqPlan& p, const int32_t* ptr,
+                          const int32_t* rows, int h_q, int h_kv, int d, int block_size, float* dqacc, bf16* dk,
+                          bf16* dv, int32_t* status, cudaStream_t st) {
 #define MOBA_BWD_TC(DD, BB)                                                                                  \
   do {                                                                                                       \
     const size_t smem = BwdTcLayout<DD, BB>::BYTES + 1024;                                                   \
@@ -350,7 +365,7 @@ cudaError_t launch_bwd_tc(const bf16* q, const bf16* k, const bf16* v, const bf1
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);     \
     if (e != cudaSuccess) return e;                                                                          \
     if (p.nb_max == 0) return cudaSuccess;                                                                   \
-    kern<<<dim3(p.nb_max, h_kv), kThreads, smem, st>>>(q, k, v, dout, lse, dsum, p.cu, p.blk_off, p.batch,   \
+    kern<<<dim3(p.nb_max, h_kv), kThreads, smem, st>>>(tm_q, k, v, tm_do, lse, dsum, p.cu, p.blk_off, p.batch, \
                                                        p.nb_max, h_q, h_kv, ptr, rows, dqacc, dk, dv, status); \
     return cudaGetLastError();                                                                               \
   } while (0)

@@ -84,12 +84,13 @@ cudaError_t launch_bwd_attn(const bf16* q, const bf16* k, const bf16* v, const b
                             float* dqacc, bf16* dk, bf16* dv, cudaStream_t st);
 
 // tcgen05 backward attention (dK, dV written; dQ added into dqacc); the
-// shapes it covers (d, B) = (64, 32), (128, 32), (128, 64).
+// shapes it covers (d, B) = (64, 32), (128, 32), (128, 64); tm_q / tm_do are
+// make_row_map over q and dout as T*H_q rows.
 bool bwd_tc_supported(int d, int block_size);
-cudaError_t launch_bwd_tc(const bf16* q, const bf16* k, const bf16* v, const bf16* dout, const float* lse,
-                          const float* dsum, const SeqPlan& p, const int32_t* ptr, const int32_t* rows, int h_q,
-                          int h_kv, int d, int block_size, float* dqacc, bf16* dk, bf16* dv, int32_t* status,
-                          cudaStream_t st);
+cudaError_t launch_bwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const CUtensorMap& tm_do,
+                          const float* lse, const float* dsum, const SeqPlan& p, const int32_t* ptr,
+                          const int32_t* rows, int h_q, int h_kv, int d, int block_size, float* dqacc, bf16* dk,
+                          bf16* dv, int32_t* status, cudaStream_t st);
 
 cudaError_t launch_bwd_dq(const float* dqacc, int n, bf16* dq, cudaStream_t st);
 

@@ -327,10 +327,12 @@ int moba_backward(const void* q, const void* k, const void* v, const void* out, 
                                 b.dqacc, st));
   STAGE_END(MOBA_STAGE_BWD_PRE);
   STAGE_BEGIN(MOBA_STAGE_BWD_ATTN);
-  if (moba::bwd_tc_supported(d, shape->block_size)) {
-    MOBA_TRY(moba::launch_bwd_tc(static_cast<const bf16*>(q), static_cast<const bf16*>(k),
-                                 static_cast<const bf16*>(v), static_cast<const bf16*>(dout), lse, b.dsum, plan, ptr,
-                                 rows, hq, hkv, d, shape->block_size, b.dqacc, static_cast<bf16*>(dk),
+  CUtensorMap tm_q, tm_do;
+  if (moba::bwd_tc_supported(d, shape->block_size) &&
+      moba::make_row_map(&tm_q, q, (unsigned long long)T * hq, d) == cudaSuccess &&
+      moba::make_row_map(&tm_do, dout, (unsigned long long)T * hq, d) == cudaSuccess) {
+    MOBA_TRY(moba::launch_bwd_tc(tm_q, static_cast<const bf16*>(k), static_cast<const bf16*>(v), tm_do, lse, b.dsum,
+                                 plan, ptr, rows, hq, hkv, d, shape->block_size, b.dqacc, static_cast<bf16*>(dk),
                                  static_cast<bf16*>(dv), b.plan.status, st));
   } else {
     MOBA_TRY(moba::launch_bwd_attn(static_cast<const bf16*>(q), static_cast<const bf16*>(k),
