@@ -8,121 +8,154 @@
 //    Formale": k'_t = k_t + SiLU(sum_{l=0}^{W-1} W_l (.) k_{t-l}), one filter
 //    per channel, causal (left zero padding at the sequence start).
 //
-// Eight threads per (global block, KV head), each owning 8 channels: a
-// thread walks the block's rows in order with 16-byte loads (the 8 threads of
-// a block read one 128/256-byte row segment together), keeps the previous
-// W-1 rows of its channels in registers for the conv, writes k' and sums the
-// (converted) keys itself, so no shared memory and no barrier are needed.
-// The sum runs in ascending token order in fp32 and is divided by the block's
-// token count.  HBM-bound: algorithmic bytes per block = B*D*2 read
-// (+ B*D*2 written with conv) + centroid outputs.
+// One CTA per (global key block, group of KV heads) with one thread per
+// channel (256 channels: 4 heads at d = 64, 2 at d = 128).  The block's rows
+// (plus the W-1 rows before it, zero outside the sequence) are staged in
+// shared memory with 16-byte cp.async copies of whole contiguous row
+// segments; each thread then walks its channel down the rows with the W taps
+// and the last W-1 keys in registers, writes k' into a shared output tile
+// (stored back with 16-byte coalesced stores) and sums the stored bf16 keys
+// in ascending token order (fp32), dividing by the block's token count.
+// HBM-bound: B*d*2 bytes read per (block, head), the same written with conv.
 #include "common.cuh"
 #include "launch.h"
 
 namespace moba {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;   // channels per CTA
 constexpr int kMaxWidth = 8;
+constexpr int kMaxBlock = 128;
+
+template <int D, int W, int BLK>
+struct CcLayout {
+  static constexpr int HG = kThreads / D;           // heads per CTA
+  static constexpr int SEG = HG * D;                // channels (bf16) per staged row
+  static constexpr int PRE = W > 1 ? W - 1 : 0;     // rows staged before the block
+  static constexpr int ROWS = BLK + PRE;
+  static constexpr uint32_t IN_BYTES = ROWS * SEG * 2;
+  static constexpr uint32_t OUT_BYTES = W > 0 ? BLK * SEG * 2 : 0;
+  static constexpr uint32_t BYTES = IN_BYTES + OUT_BYTES;
+};
+
+template <int D, int W, int BLK>
+__global__ void __launch_bounds__(kThreads)
+conv_centroid_kernel(const bf16* __restrict__ k, const float* __restrict__ conv_w, const int32_t* __restrict__ cu,
+                     const int32_t* __restrict__ blk_off, int batch, int nb_max, int h_kv, bf16* __restrict__ k_out,
+                     float* __restrict__ cent, bf16* __restrict__ cent_hi, bf16* __restrict__ cent_lo) {
+  using Ly = CcLayout<D, W, BLK>;
+  extern __shared__ __align__(16) unsigned char smem[];
+  bf16* in = reinterpret_cast<bf16*>(smem);                    // [ROWS][SEG]
+  bf16* outt = reinterpret_cast<bf16*>(smem + Ly::IN_BYTES);   // [BLK][SEG]
+
+  const int gb = blockIdx.x;
+  const int h0 = blockIdx.y * Ly::HG;
+  if (gb >= __ldg(blk_off + batch)) return;
+  const int s = upper_seq(blk_off, batch, gb);
+  const int seq0 = __ldg(cu + s), seq1 = __ldg(cu + s + 1);
+  const int t0 = seq0 + (gb - __ldg(blk_off + s)) * BLK;
+  const int t1 = min(t0 + BLK, seq1);
+  const int tid = threadIdx.x;
+  const size_t row_stride = (size_t)h_kv * D;
+  const int nh = min(Ly::HG, h_kv - h0);                       // heads of this CTA that exist
+
+  // ---- stage rows t0-PRE .. t0+BLK-1 (zero outside [seq0, t1))
+  constexpr int CPR = Ly::SEG / 8;                             // 16-byte chunks per staged row
+  for (int i = tid; i < Ly::ROWS * CPR; i += kThreads) {
+    const int r = i / CPR, c = i % CPR;
+    const int t = t0 - Ly::PRE + r;
+    const bool ok = t >= seq0 && t < t1 && c * 8 < nh * D;
+    const size_t off = ok ? (size_t)t * row_stride + (size_t)h0 * D + c * 8 : 0;
+    cp_async16_zfill(in + r * Ly::SEG + c * 8, k + off, ok);
+  }
+  cp_async_commit();
+  const int ch = tid;                                          // channel within the segment
+  const int h = h0 + ch / D, c = ch % D;
+  float w[W > 0 ? W : 1];
+#pragma unroll
+  for (int l = 0; l < W; ++l) w[l] = h < h_kv ? __ldg(conv_w + ((size_t)h * D + c) * W + l) : 0.f;
+  cp_async_wait<0>();
+  __syncthreads();
+
+  const int n = t1 - t0;
+  float acc = 0.f;
+  if constexpr (W == 0) {
+    for (int r = 0; r < n; ++r) acc += __bfloat162float(in[r * Ly::SEG + ch]);
+  } else {
+    // win[l] = k_{t-1-l}
+    float win[W > 1 ? W - 1 : 1];
+#pragma unroll
+    for (int l = 0; l < W - 1; ++l) win[l] = __bfloat162float(in[(Ly::PRE - 1 - l) * Ly::SEG + ch]);
+#pragma unroll 4
+    for (int r = 0; r < BLK; ++r) {
+      const float cur = __bfloat162float(in[(Ly::PRE + r) * Ly::SEG + ch]);
+      float x = w[0] * cur;
+#pragma unroll
+      for (int l = 1; l < W; ++l) x = fmaf(w[l], win[l - 1], x);
+      const bf16 y = __float2bfloat16_rn(cur + __fdividef(x, 1.f + __expf(-x)));  // k + SiLU(x)
+      outt[r * Ly::SEG + ch] = y;
+      if (r < n) acc += __bfloat162float(y);  // the centroid averages the stored bf16 keys
+#pragma unroll
+      for (int l = W - 2; l > 0; --l) win[l] = win[l - 1];
+      if (W > 1) win[0] = cur;
+    }
+    __syncthreads();
+    for (int i = tid; i < n * CPR; i += kThreads) {
+      const int r = i / CPR, cc = i % CPR;
+      if (cc * 8 < nh * D)
+        *reinterpret_cast<uint4*>(k_out + (size_t)(t0 + r) * row_stride + (size_t)h0 * D + cc * 8) =
+            *reinterpret_cast<const uint4*>(outt + r * Ly::SEG + cc * 8);
+    }
+  }
+  if (h < h_kv) {
+    const float cv = acc / (float)n;
+    const bf16 hb = __float2bfloat16_rn(cv);
+    const size_t o = ((size_t)h * nb_max + gb) * D + c;
+    cent[o] = cv;
+    cent_hi[o] = hb;
+    cent_lo[o] = __float2bfloat16_rn(cv - __bfloat162float(hb));
+  }
+}
+
+template <int D, int W>
+cudaError_t launch_cc_w(const bf16* k, const float* conv_w, const SeqPlan& p, int h_kv, int block_size, bf16* k_out,
+                        float* cent, bf16* cent_hi, bf16* cent_lo, cudaStream_t st) {
+  const dim3 grid(p.nb_max, (h_kv + kThreads / D - 1) / (kThreads / D));
+#define MOBA_CC(BB)                                                                                      \
+  {                                                                                                      \
+    const size_t smem = CcLayout<D, W, BB>::BYTES;                                                       \
+    auto kern = conv_centroid_kernel<D, W, BB>;                                                          \
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    if (e != cudaSuccess) return e;                                                                      \
+    kern<<<grid, kThreads, smem, st>>>(k, conv_w, p.cu, p.blk_off, p.batch, p.nb_max, h_kv, k_out, cent,  \
+                                       cent_hi, cent_lo);                                                \
+    return cudaGetLastError();                                                                           \
+  }
+  switch (block_size) {
+    case 16: MOBA_CC(16);
+    case 32: MOBA_CC(32);
+    case 64: MOBA_CC(64);
+    case 128: MOBA_CC(128);
+  }
+#undef MOBA_CC
+  return cudaErrorInvalidValue;
+}
 
 template <int D>
-__global__ void __launch_bounds__(kThreads)
-conv_centroid_kernel(const bf16* __restrict__ k, const float* __restrict__ conv_w, int width,
-                     const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch,
-                     int nb_max, int h_kv, int block_size, bf16* __restrict__ k_out,
-                     float* __restrict__ cent, bf16* __restrict__ cent_hi, bf16* __restrict__ cent_lo) {
-  constexpr int TPB = D / 8;  // threads per block (8 channels each)
-  const long long gtid = (long long)blockIdx.x * kThreads + threadIdx.x;
-  const int c8 = (int)(gtid % TPB);
-  const long long bidx = gtid / TPB;
-  const int h = (int)(bidx / nb_max);
-  const int gb = (int)(bidx % nb_max);
-  if (h >= h_kv || gb >= __ldg(blk_off + batch)) return;
-  const int s = upper_seq(blk_off, batch, gb);
-  const int j = gb - __ldg(blk_off + s);
-  const int seq0 = __ldg(cu + s);
-  const int t0 = seq0 + j * block_size;
-  const int t1 = min(t0 + block_size, __ldg(cu + s + 1));
-  const size_t row_stride = (size_t)h_kv * D;
-  const bf16* kh = k + (size_t)h * D + c8 * 8;
-
-  float acc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-
-  if (width == 0) {
-#pragma unroll 4
-    for (int t = t0; t < t1; ++t) {
-      float f[8];
-      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kh + (size_t)t * row_stride)), f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += f[i];
-    }
-  } else {
-    float w[kMaxWidth][8];
-#pragma unroll
-    for (int l = 0; l < kMaxWidth; ++l)
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        w[l][i] = l < width ? __ldg(conv_w + ((size_t)h * D + c8 * 8 + i) * width + l) : 0.f;
-    // win[l] holds k_{t-1-l} (zero before the sequence start)
-    float win[kMaxWidth - 1][8];
-#pragma unroll
-    for (int l = 0; l < kMaxWidth - 1; ++l) {
-      const int tp = t0 - 1 - l;
-      if (l + 1 < width && tp >= seq0) {
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kh + (size_t)tp * row_stride)), win[l]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) win[l][i] = 0.f;
-      }
-    }
-    bf16* ko = k_out + (size_t)h * D + c8 * 8;
-#pragma unroll 2
-    for (int t = t0; t < t1; ++t) {
-      float cur[8], x[8];
-      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kh + (size_t)t * row_stride)), cur);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = w[0][i] * cur[i];
-#pragma unroll
-      for (int l = 1; l < kMaxWidth; ++l)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = fmaf(w[l][i], win[l - 1][i], x[i]);
-      float y[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) y[i] = cur[i] + x[i] / (1.f + expf(-x[i]));
-      const uint4 packed = f32_to_bf16x8(y);
-      *reinterpret_cast<uint4*>(ko + (size_t)t * row_stride) = packed;
-      float yr[8];
-      bf16x8_to_f32(packed, yr);  // the centroid averages the stored bf16 keys
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += yr[i];
-#pragma unroll
-      for (int l = kMaxWidth - 2; l > 0; --l)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) win[l][i] = win[l - 1][i];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) win[0][i] = cur[i];
-    }
+cudaError_t launch_cc_d(const bf16* k, const float* conv_w, int conv_width, const SeqPlan& p, int h_kv,
+                        int block_size, bf16* k_out, float* cent, bf16* cent_hi, bf16* cent_lo, cudaStream_t st) {
+  switch (conv_width) {
+    case 0: return launch_cc_w<D, 0>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
+    case 1: return launch_cc_w<D, 1>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
+    case 2: return launch_cc_w<D, 2>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
+    case 3: return launch_cc_w<D, 3>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
+    case 4: return launch_cc_w<D, 4>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
+    case 5: return launch_cc_w<D, 5>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
+    case 6: return launch_cc_w<D, 6>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
+    case 7: return launch_cc_w<D, 7>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
+    case 8: return launch_cc_w<D, 8>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
   }
-
-  const float inv = 1.f / (float)(t1 - t0);
-  float c[8], lo[8];
-  bf16 hb[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    c[i] = acc[i] * inv;
-    hb[i] = __float2bfloat16_rn(c[i]);
-    lo[i] = c[i] - __bfloat162float(hb[i]);
-  }
-  const size_t o = ((size_t)h * nb_max + gb) * D + c8 * 8;
-  reinterpret_cast<float4*>(cent + o)[0] = make_float4(c[0], c[1], c[2], c[3]);
-  reinterpret_cast<float4*>(cent + o)[1] = make_float4(c[4], c[5], c[6], c[7]);
-  float hf[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) hf[i] = __bfloat162float(hb[i]);
-  *reinterpret_cast<uint4*>(cent_hi + o) = f32_to_bf16x8(hf);
-  *reinterpret_cast<uint4*>(cent_lo + o) = f32_to_bf16x8(lo);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -130,17 +163,10 @@ conv_centroid_kernel(const bf16* __restrict__ k, const float* __restrict__ conv_
 cudaError_t launch_conv_centroid(const bf16* k, const float* conv_w, int conv_width, const SeqPlan& p,
                                  int h_kv, int d, int block_size, bf16* k_out, float* cent,
                                  bf16* cent_hi, bf16* cent_lo, cudaStream_t st) {
-  if (conv_width > kMaxWidth) return cudaErrorInvalidValue;
-  const long long threads = (long long)p.nb_max * h_kv * (d / 8);
-  const int grid = (int)((threads + kThreads - 1) / kThreads);
-  if (grid == 0) return cudaSuccess;
-  if (d == 64)
-    conv_centroid_kernel<64><<<grid, kThreads, 0, st>>>(k, conv_w, conv_width, p.cu, p.blk_off, p.batch, p.nb_max,
-                                                        h_kv, block_size, k_out, cent, cent_hi, cent_lo);
-  else
-    conv_centroid_kernel<128><<<grid, kThreads, 0, st>>>(k, conv_w, conv_width, p.cu, p.blk_off, p.batch, p.nb_max,
-                                                         h_kv, block_size, k_out, cent, cent_hi, cent_lo);
-  return cudaGetLastError();
+  if (conv_width < 0 || conv_width > kMaxWidth || block_size > kMaxBlock) return cudaErrorInvalidValue;
+  if (p.nb_max == 0 || h_kv == 0) return cudaSuccess;
+  if (d == 64) return launch_cc_d<64>(k, conv_w, conv_width, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
+  return launch_cc_d<128>(k, conv_w, conv_width, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
 }
 
 }  // namespace moba
