@@ -34,7 +34,6 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kScanThreads = 1024;
 constexpr int kChunkTokens = 1024;
-constexpr int kBatch = 8;  // picks per thread with their loads in flight together
 constexpr int kMaxSmemBuckets = 16384;  // 64 KB of shared-memory counters
 
 // Returns the bucket of pick `e` (row * topk + slot) or -1 if the slot is
@@ -114,36 +113,55 @@ fill_kernel(const int32_t* __restrict__ sel_idx, long long npicks, int topk, int
 }
 
 // ---- shared-memory privatised path
+//
+// A CTA owns the picks of one (chunk of kChunkTokens tokens, KV head): one
+// thread per query row (token, query head of the group) at a time, which
+// locates its sequence once and then walks the row's topk picks (16-byte
+// loads), so the per-pick work is a load, a range check and one
+// shared-memory atomic.
 
-// Pick i of chunk (tokens [ta, ta + kChunkTokens)) of KV head kvh: its
-// position in sel_idx, or -1 past the chunk / outside every sequence.
-// Also returns the pick's token and query row id.
-__device__ __forceinline__ long long chunk_pick_pos(int i, int n, int ta, int kvh, int group, int topk, int h_q,
-                                                    int seq_end, int& t, int& row) {
-  if (i >= n) return -1;
-  const int per_tok = group * topk;
-  t = ta + i / per_tok;
-  if (t >= seq_end) return -1;
-  const int rem = i - (t - ta) * per_tok;
-  row = t * h_q + kvh * group + rem / topk;
-  return (long long)row * topk + rem % topk;
+// For query row `r` of the chunk (ta: first token): its row id, its
+// sequence's first global block and its own block; false past the chunk or
+// outside every sequence.
+__device__ __forceinline__ bool chunk_row(int r, int ntok, int ta, int kvh, int group, int h_q, int block_size,
+                                          const int32_t* cu, const int32_t* blk_off, int batch, int seq_end,
+                                          int& row, int& base, int& own) {
+  if (r >= ntok * group) return false;
+  const int t = ta + r / group;
+  if (t >= seq_end) return false;
+  row = t * h_q + kvh * group + r % group;
+  const int s = upper_seq(cu, batch, t);
+  base = __ldg(blk_off + s);
+  own = (t - __ldg(cu + s)) / block_size;
+  return true;
 }
 
-// Local bucket (blk_off[s] + j) of the pick at `e` holding block j, or -1 if
-// the slot is empty or invalid (invalid entries raise kStatusBadSelIdx).
-__device__ __forceinline__ int chunk_pick_bucket(long long e, int t, int j, int block_size, const int32_t* cu,
-                                                 const int32_t* blk_off, int batch, int32_t* status) {
-  if (e < 0) return -1;
-  if (j < 0) {
-    if (j != -1) set_status(status, kStatusBadSelIdx);
-    return -1;
+// Calls f(m, j) for the valid picks of a row (j in [0, own]); invalid
+// entries are skipped (and raise kStatusBadSelIdx when `kReport`).
+template <bool kReport, typename F>
+__device__ __forceinline__ void for_row_picks(const int32_t* __restrict__ sel_idx, int row, int topk, int own,
+                                              int32_t* status, F&& f) {
+  const int32_t* p = sel_idx + (size_t)row * topk;
+  auto one = [&](int m, int j) {
+    if (j < 0) {
+      if (kReport && j != -1) set_status(status, kStatusBadSelIdx);
+    } else if (j > own) {
+      if (kReport) set_status(status, kStatusBadSelIdx);
+    } else {
+      f(m, j);
+    }
+  };
+  int m = 0;
+  if ((topk & 3) == 0) {  // rows start 16-byte aligned
+    for (; m < topk; m += 4) {
+      const int4 v = __ldg(reinterpret_cast<const int4*>(p + m));
+      one(m, v.x);
+      one(m + 1, v.y);
+      one(m + 2, v.z);
+      one(m + 3, v.w);
+    }
   }
-  const int s = upper_seq(cu, batch, t);
-  if (j > (t - __ldg(cu + s)) / block_size) {
-    set_status(status, kStatusBadSelIdx);
-    return -1;
-  }
-  return __ldg(blk_off + s) + j;
+  for (; m < topk; ++m) one(m, __ldg(p + m));
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -155,21 +173,12 @@ chunk_count_kernel(const int32_t* __restrict__ sel_idx, int total_tokens, int to
   for (int b = threadIdx.x; b < nb_max; b += kThreads) hist[b] = 0;
   __syncthreads();
   const int ta = c * kChunkTokens;
-  const int n = max(0, min(kChunkTokens, total_tokens - ta)) * group * topk;
+  const int ntok = max(0, min(kChunkTokens, total_tokens - ta));
   const int seq_end = __ldg(cu + batch);
-  for (int i0 = threadIdx.x; i0 < n; i0 += kThreads * kBatch) {
-    long long e[kBatch];
-    int j[kBatch], t[kBatch], row[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      e[u] = chunk_pick_pos(i0 + u * kThreads, n, ta, kvh, group, topk, h_q, seq_end, t[u], row[u]);
-      j[u] = e[u] >= 0 ? __ldg(sel_idx + e[u]) : -1;
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int lb = chunk_pick_bucket(e[u], t[u], j[u], block_size, cu, blk_off, batch, status);
-      if (lb >= 0) atomicAdd(hist + lb, 1);
-    }
+  for (int r = threadIdx.x; r < ntok * group; r += kThreads) {
+    int row, base, own;
+    if (!chunk_row(r, ntok, ta, kvh, group, h_q, block_size, cu, blk_off, batch, seq_end, row, base, own)) continue;
+    for_row_picks<true>(sel_idx, row, topk, own, status, [&](int, int j) { atomicAdd(hist + base + j, 1); });
   }
   __syncthreads();
   int32_t* dst = chunk_cnt + ((size_t)kvh * nchunks + c) * nb_max;
@@ -201,26 +210,18 @@ chunk_fill_kernel(const int32_t* __restrict__ sel_idx, int total_tokens, int top
   extern __shared__ int32_t cursor[];
   const int c = blockIdx.x, kvh = blockIdx.y;
   const int32_t* src = chunk_cnt + ((size_t)kvh * nchunks + c) * nb_max;
-  const int32_t* base = ptr + (size_t)kvh * nb_max;
-  for (int b = threadIdx.x; b < nb_max; b += kThreads) cursor[b] = __ldg(base + b) + __ldg(src + b);
+  const int32_t* bptr = ptr + (size_t)kvh * nb_max;
+  for (int b = threadIdx.x; b < nb_max; b += kThreads) cursor[b] = __ldg(bptr + b) + __ldg(src + b);
   __syncthreads();
   const int ta = c * kChunkTokens;
-  const int n = max(0, min(kChunkTokens, total_tokens - ta)) * group * topk;
+  const int ntok = max(0, min(kChunkTokens, total_tokens - ta));
   const int seq_end = __ldg(cu + batch);
-  for (int i0 = threadIdx.x; i0 < n; i0 += kThreads * kBatch) {
-    long long e[kBatch];
-    int j[kBatch], t[kBatch], row[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      e[u] = chunk_pick_pos(i0 + u * kThreads, n, ta, kvh, group, topk, h_q, seq_end, t[u], row[u]);
-      j[u] = e[u] >= 0 ? __ldg(sel_idx + e[u]) : -1;
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      // invalid entries were reported by the count pass
-      const int lb = chunk_pick_bucket(e[u], t[u], j[u], block_size, cu, blk_off, batch, status);
-      if (lb >= 0) rows[atomicAdd(cursor + lb, 1)] = row[u];
-    }
+  // (invalid entries were reported by the count pass)
+  for (int r = threadIdx.x; r < ntok * group; r += kThreads) {
+    int row, base, own;
+    if (!chunk_row(r, ntok, ta, kvh, group, h_q, block_size, cu, blk_off, batch, seq_end, row, base, own)) continue;
+    for_row_picks<false>(sel_idx, row, topk, own, status,
+                         [&](int, int j) { rows[atomicAdd(cursor + base + j, 1)] = row; });
   }
 }
 
