@@ -395,8 +395,12 @@ def run_ours(args):
 
         dev_in = [{n: torch.empty_like(g[n]) for n in names_in} for _ in range(2)]
         dev_out = [out_set() for _ in range(2)]
-        host_out = [{n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in o.items()} for o in dev_out]
-        d2h = sum(t.numel() * t.element_size() for t in dev_out[0].values())
+        # The step's results: O, LSE, dQ, dV and the key gradients the caller
+        # holds (dK and dW of the original keys when the conv is applied; dK'
+        # is then an intermediate that stays on the device).
+        results = ["out", "lse", "dq", "dv"] + (["dk_in", "dw"] if conv_w is not None else ["dk"])
+        host_out = [{n: torch.empty(o[n].shape, dtype=o[n].dtype, pin_memory=True) for n in results} for o in dev_out]
+        d2h = sum(dev_out[0][n].numel() * dev_out[0][n].element_size() for n in results)
         s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         ev_in = [torch.cuda.Event() for _ in range(2)]
         ev_fwd = [torch.cuda.Event() for _ in range(2)]
@@ -434,7 +438,7 @@ def run_ours(args):
                 ho["lse"].copy_(do_["lse"], non_blocking=True)
             s_out.wait_event(ev_cmp[b])
             with torch.cuda.stream(s_out):
-                for n in do_:
+                for n in results:
                     if n not in ("out", "lse"):
                         ho[n].copy_(do_[n], non_blocking=True)
                 ev_out[b].record(s_out)
@@ -444,7 +448,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        ne = max(3, min(2 * args.steps, 10))
+        ne = max(3, min(2 * args.steps, 20))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(s_in)
         for i in range(ne):
