@@ -301,3 +301,50 @@ def test_rows_far_above_the_reference_take_the_exact_path(dev, d, B):
         for t, hh in bad:
             o_ref[t, hh], lse_ref[t, hh] = o2[t, hh], l2[t, hh]
     pu.check_o_lse(o_g, lse_g, o_ref, lse_ref, "overflow_d%d_B%d" % (d, B))
+
+
+def test_forward_backward_replay_from_a_cuda_graph(dev):
+    # The entry points allocate nothing, never synchronise and take the
+    # stream, so a whole forward + backward (+ key-conv backward) step can be
+    # captured once and replayed; the replay must give what eager calls give.
+    case = ((2048,), 2, 2, 64, 32, 8, 4)
+    w, x = _inputs(case)
+    g = _gpu(x, dev)
+    B, k = w.block_size, w.topk
+    shape = moba.shape_of(g["q"], g["k"], g["cu_seqlens"], B, k)
+    ws_f = moba.alloc_workspace(moba.fwd_workspace_size(shape), dev)
+    ws_b = moba.alloc_workspace(moba.bwd_workspace_size(shape), dev)
+    out, lse = torch.empty_like(g["q"]), torch.empty(g["q"].shape[:2], dtype=torch.float32, device=dev)
+    sel = torch.empty(g["q"].shape[:2] + (k,), dtype=torch.int32, device=dev)
+    kc = torch.empty_like(g["k"])
+    dq, dk, dv = torch.empty_like(g["q"]), torch.empty_like(g["k"]), torch.empty_like(g["v"])
+    dk_in, dw = torch.empty_like(g["k"]), torch.empty_like(g["conv_w"])
+
+    def step():
+        _, _, _, ku = moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], B, k, conv_w=g["conv_w"],
+                                   workspace=ws_f, out=out, lse=lse, sel_idx=sel, k_conv=kc)
+        moba.backward(g["q"], ku, g["v"], out, lse, g["dout"], sel, g["cu_seqlens"], B, workspace=ws_b,
+                      dq=dq, dk=dk, dv=dv, fwd_workspace=ws_f)
+        moba.key_conv_backward(g["k"], g["conv_w"], g["cu_seqlens"], B, dk, workspace=ws_b, dk=dk_in, dw=dw)
+
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        step()                                   # eager, on the capture stream
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize()
+    eager = [t.clone() for t in (out, lse, sel, dq, dv, dk_in, dw)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        step()
+    for t in (out, lse, dq, dv, dk_in, dw):
+        t.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert moba.check_status(ws_f) == 0 and moba.check_status(ws_b) == 0
+    got = (out, lse, sel, dq, dv, dk_in, dw)
+    assert torch.equal(got[2], eager[2])
+    for a, b in zip(got, eager):
+        # fp32 reductions may add in another order: compare to bf16 resolution
+        assert (a.float() - b.float()).abs().max().item() <= 2e-2 * max(1.0, b.float().abs().max().item())
+    del graph
