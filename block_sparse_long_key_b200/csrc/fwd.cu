@@ -60,9 +60,10 @@ __global__ void __launch_bounds__(kThreads)
 fwd_attn_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                 const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch, int nb_max,
                 int h_q, int h_kv, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
-                const float* __restrict__ mref, float* __restrict__ oacc, int32_t* __restrict__ flag) {
+                const float* __restrict__ mref, float* __restrict__ oacc, float* __restrict__ lacc,
+                int32_t* __restrict__ flag) {
   constexpr int KC = BLK < 64 ? BLK : 64;  // keys per register chunk
-  constexpr int OS = oacc_stride(D);       // accumulator row: O (D), l, padding
+  constexpr int OS = oacc_stride(D);       // accumulator row: O (D); l in lacc
   constexpr unsigned FULL = 0xffffffffu;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   FwdSmem<D, BLK>& sm = *reinterpret_cast<FwdSmem<D, BLK>*>(smem_raw);
@@ -234,11 +235,11 @@ fwd_attn_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
     }
     if (q4 == 0) {
       if (row0 >= 0) {
-        atomicAdd(oacc + (size_t)row0 * OS + D, l0);
+        atomicAdd(lacc + row0, l0);
         if (mx0 - mr0 > kOverflowLog2) flag[row0] = 1;
       }
       if (row1 >= 0) {
-        atomicAdd(oacc + (size_t)row1 * OS + D, l1);
+        atomicAdd(lacc + row1, l1);
         if (mx1 - mr1 > kOverflowLog2) flag[row1] = 1;
       }
     }
@@ -251,9 +252,9 @@ fwd_attn_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
 }
 
 // O = acc / l (bf16), LSE = M + log l; flagged rows are queued instead.
-// Accumulator rows are oacc_stride(D) floats: O, then l, then padding.
+// Accumulator rows are oacc_stride(D) floats of O; l is in its own array.
 __global__ void __launch_bounds__(256)
-fwd_finalize_kernel(const float* __restrict__ oacc, const float* __restrict__ mref,
+fwd_finalize_kernel(const float* __restrict__ oacc, const float* __restrict__ lacc, const float* __restrict__ mref,
                     const int32_t* __restrict__ flag, long long nchunks, int d8, bf16* __restrict__ out,
                     float* __restrict__ lse, int32_t* __restrict__ flag_list) {
   const int os = oacc_stride(d8 * 8);
@@ -268,7 +269,7 @@ fwd_finalize_kernel(const float* __restrict__ oacc, const float* __restrict__ mr
       continue;
     }
     const float* acc = oacc + row * os;
-    const float l = __ldg(acc + d8 * 8);
+    const float l = __ldg(lacc + row);
     const float inv = 1.f / l;
     const float4* src = reinterpret_cast<const float4*>(acc + c * 8);
     const float4 a = __ldg(src), b = __ldg(src + 1);
@@ -331,7 +332,7 @@ fwd_fallback_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, cons
 
 template <int D, int BLK>
 cudaError_t launch_fwd_t(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p, const int32_t* ptr,
-                         const int32_t* rows, const float* mref, int h_q, int h_kv, float* oacc,
+                         const int32_t* rows, const float* mref, int h_q, int h_kv, float* oacc, float* lacc,
                          int32_t* flag, cudaStream_t st) {
   const size_t smem = sizeof(FwdSmem<D, BLK>);
   auto kern = fwd_attn_kernel<D, BLK>;
@@ -340,7 +341,7 @@ cudaError_t launch_fwd_t(const bf16* q, const bf16* k, const bf16* v, const SeqP
   if (p.nb_max == 0) return cudaSuccess;
   dim3 grid(p.nb_max, h_kv);
   kern<<<grid, kThreads, smem, st>>>(q, k, v, p.cu, p.blk_off, p.batch, p.nb_max, h_q, h_kv, ptr, rows, mref,
-                                     oacc, flag);
+                                     oacc, lacc, flag);
   return cudaGetLastError();
 }
 
@@ -348,8 +349,8 @@ cudaError_t launch_fwd_t(const bf16* q, const bf16* k, const bf16* v, const SeqP
 
 cudaError_t launch_fwd_attn(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p, const int32_t* ptr,
                             const int32_t* rows, const float* mref, int h_q, int h_kv, int d, int block_size,
-                            float* oacc, int32_t* flag, cudaStream_t st) {
-#define MOBA_FWD(DD, BB) return launch_fwd_t<DD, BB>(q, k, v, p, ptr, rows, mref, h_q, h_kv, oacc, flag, st)
+                            float* oacc, float* lacc, int32_t* flag, cudaStream_t st) {
+#define MOBA_FWD(DD, BB) return launch_fwd_t<DD, BB>(q, k, v, p, ptr, rows, mref, h_q, h_kv, oacc, lacc, flag, st)
   if (d == 64) {
     switch (block_size) {
       case 16: MOBA_FWD(64, 16);
@@ -369,14 +370,14 @@ cudaError_t launch_fwd_attn(const bf16* q, const bf16* k, const bf16* v, const S
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_fwd_finalize(const float* oacc, const float* mref, const int32_t* flag, int nrows, int d,
+cudaError_t launch_fwd_finalize(const float* oacc, const float* lacc, const float* mref, const int32_t* flag, int nrows, int d,
                                 bf16* out, float* lse, int32_t* flag_list, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(flag_list, 0, sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
   const long long nchunks = (long long)nrows * (d / 8);
   if (nchunks == 0) return cudaSuccess;
   const int grid = (int)std::min<long long>((nchunks + 255) / 256, 148LL * 32);
-  fwd_finalize_kernel<<<grid, 256, 0, st>>>(oacc, mref, flag, nchunks, d / 8, out, lse, flag_list);
+  fwd_finalize_kernel<<<grid, 256, 0, st>>>(oacc, lacc, mref, flag, nchunks, d / 8, out, lse, flag_list);
   return cudaGetLastError();
 }
 

@@ -19,8 +19,8 @@
 //   4. One thread issues O = P V_j (M = 128, N = d, K = B; V_j read
 //      N-major) into the columns S used.
 //   5. Each thread reads its O row and adds it, and l, to the query's fp32
-//      accumulator row [O | l | pad] with 16-byte vector reductions (lane
-//      pairs cover whole 32-byte sectors).
+//      accumulator row (O, d floats; l in its own array) with 16-byte
+//      vector reductions (lane pairs cover whole 32-byte sectors).
 // The merge of a query's k blocks is therefore a plain sum; finalize divides
 // by l.  A CTA needs ~33 KB of shared memory and 64 TMEM columns at d = 64,
 // so several share an SM and overlap their phases.  Every mbarrier wait is
@@ -69,7 +69,8 @@ __global__ void __launch_bounds__(kThreads)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__ k, const bf16* __restrict__ v,
               const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch, int nb_max,
               int h_q, int h_kv, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
-              const float* __restrict__ mref, float* __restrict__ oacc, int32_t* __restrict__ flag,
+              const float* __restrict__ mref, float* __restrict__ oacc, float* __restrict__ lacc,
+              int32_t* __restrict__ flag,
               int32_t* __restrict__ status) {
   using Ly = FwdTcLayout<D, BLK>;
   constexpr int OS = oacc_stride(D);
@@ -230,7 +231,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
     }
     tc::fence_after_sync();
     if (rid >= 0) {
-      atomicAdd(oacc + (size_t)rid * OS + D, l);
+      atomicAdd(lacc + rid, l);
       if (mx - mr_c > kOverflowLog2) flag[rid] = 1;
     }
     const int prow = __shfl_xor_sync(0xffffffffu, rid, 1);  // the lane pair's other row
@@ -297,7 +298,8 @@ bool fwd_tc_supported(int d, int block_size) {
 
 cudaError_t launch_fwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const SeqPlan& p,
                           const int32_t* ptr, const int32_t* rows, const float* mref, int h_q, int h_kv, int d,
-                          int block_size, float* oacc, int32_t* flag, int32_t* status, cudaStream_t st) {
+                          int block_size, float* oacc, float* lacc, int32_t* flag, int32_t* status,
+                          cudaStream_t st) {
 #define MOBA_FWD_TC(DD, BB)                                                                                   \
   do {                                                                                                        \
     const size_t smem = FwdTcLayout<DD, BB>::BYTES + 1024;                                                    \
@@ -306,7 +308,7 @@ cudaError_t launch_fwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v,
     if (e != cudaSuccess) return e;                                                                           \
     if (p.nb_max == 0) return cudaSuccess;                                                                    \
     kern<<<dim3(p.nb_max, h_kv), kThreads, smem, st>>>(tm_q, k, v, p.cu, p.blk_off, p.batch, p.nb_max, h_q,   \
-                                                       h_kv, ptr, rows, mref, oacc, flag, status);            \
+                                                       h_kv, ptr, rows, mref, oacc, lacc, flag, status);            \
     return cudaGetLastError();                                                                                \
   } while (0)
   if (d == 64 && block_size == 32) MOBA_FWD_TC(64, 32);

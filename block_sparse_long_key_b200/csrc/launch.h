@@ -34,13 +34,14 @@ cudaError_t launch_conv_centroid(const bf16* k, const float* conv_w, int conv_wi
                                  bf16* cent_hi, bf16* cent_lo, cudaStream_t st);
 
 // Forward accumulator rows: O (d floats), l, 3 floats of padding.
-// Forward accumulator row: O (d floats), l, padding to a 32-byte multiple so
-// that every row starts on an L2 sector.
-__host__ __device__ constexpr int oacc_stride(int d) { return d + 8; }
+// Forward accumulator: rows of d floats (the unnormalised O, 256- or
+// 512-byte rows, so each starts on an L2 line) and, separately, one float l
+// per row.
+__host__ __device__ constexpr int oacc_stride(int d) { return d; }
 
 cudaError_t launch_route(const bf16* q, const bf16* k, const bf16* cent_hi, const bf16* cent_lo,
                          const SeqPlan& p, int h_q, int h_kv, int d, int block_size, int topk,
-                         int32_t* sel_idx, float* mref, int32_t* flag, float* oacc,
+                         int32_t* sel_idx, float* mref, int32_t* flag, float* oacc, float* lacc,
                          int32_t* status, cudaStream_t st);
 
 // chunk_cnt (optional, index_chunk_ints() int32) selects the shared-memory
@@ -53,7 +54,8 @@ cudaError_t launch_build_index(const int32_t* sel_idx, const SeqPlan& p, int h_q
 
 cudaError_t launch_fwd_attn(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p,
                             const int32_t* ptr, const int32_t* rows, const float* mref, int h_q,
-                            int h_kv, int d, int block_size, float* oacc, int32_t* flag, cudaStream_t st);
+                            int h_kv, int d, int block_size, float* oacc, float* lacc, int32_t* flag,
+                            cudaStream_t st);
 
 // Tensor map over a [nrows, d] bf16 row table (16-byte aligned base) for
 // the tile::gather4 row gathers: 64-element boxes one row high, 128-byte
@@ -65,9 +67,10 @@ cudaError_t make_row_map(CUtensorMap* map, const void* base, unsigned long long 
 bool fwd_tc_supported(int d, int block_size);
 cudaError_t launch_fwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const SeqPlan& p,
                           const int32_t* ptr, const int32_t* rows, const float* mref, int h_q, int h_kv, int d,
-                          int block_size, float* oacc, int32_t* flag, int32_t* status, cudaStream_t st);
+                          int block_size, float* oacc, float* lacc, int32_t* flag, int32_t* status,
+                          cudaStream_t st);
 
-cudaError_t launch_fwd_finalize(const float* oacc, const float* mref, const int32_t* flag, int nrows,
+cudaError_t launch_fwd_finalize(const float* oacc, const float* lacc, const float* mref, const int32_t* flag, int nrows,
                                 int d, bf16* out, float* lse, int32_t* flag_list, cudaStream_t st);
 
 cudaError_t launch_fwd_fallback(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p,

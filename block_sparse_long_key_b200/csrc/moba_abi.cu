@@ -67,7 +67,8 @@ struct FwdBufs {
   bf16* lo;
   float* mref;
   int32_t* flag;
-  float* oacc;  // rows of oacc_stride(d) floats: O, l, padding
+  float* oacc;  // rows of oacc_stride(d) floats: the unnormalised O
+  float* lacc;  // one float per row: the softmax denominator l
   int32_t* cnt;
   int32_t* ptr;
   int32_t* cursor;
@@ -88,6 +89,7 @@ FwdBufs carve_fwd(Carve& c, const moba_shape* s) {
   b.mref = c.take<float>(nrow);
   b.flag = c.take<int32_t>(nrow);
   b.oacc = c.take<float>(nrow * moba::oacc_stride(s->head_dim));
+  b.lacc = c.take<float>(nrow);
   b.cnt = c.take<int32_t>(nbk);
   b.ptr = c.take<int32_t>(nbk + 1);
   b.cursor = c.take<int32_t>(nbk);
@@ -249,7 +251,7 @@ int moba_forward(const void* q, const void* k, const void* v, const int32_t* cu_
                                       static_cast<bf16*>(k_conv_out), b.cent, b.hi, b.lo, st));
   STAGE_END(MOBA_STAGE_FWD_CENTROID);
   STAGE_BEGIN(MOBA_STAGE_FWD_ROUTE);
-  MOBA_TRY(moba::launch_route(kq, kk, b.hi, b.lo, plan, hq, hkv, d, B, topk, sel_idx, b.mref, b.flag, b.oacc,
+  MOBA_TRY(moba::launch_route(kq, kk, b.hi, b.lo, plan, hq, hkv, d, B, topk, sel_idx, b.mref, b.flag, b.oacc, b.lacc,
                               b.plan.status, st));
   STAGE_END(MOBA_STAGE_FWD_ROUTE);
   STAGE_BEGIN(MOBA_STAGE_FWD_INDEX);
@@ -259,13 +261,14 @@ int moba_forward(const void* q, const void* k, const void* v, const int32_t* cu_
   STAGE_BEGIN(MOBA_STAGE_FWD_ATTN);
   CUtensorMap tm_q;
   if (moba::fwd_tc_supported(d, B) && moba::make_row_map(&tm_q, kq, (unsigned long long)T * hq, d) == cudaSuccess)
-    MOBA_TRY(moba::launch_fwd_tc(tm_q, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.flag,
-                                 b.plan.status, st));
+    MOBA_TRY(moba::launch_fwd_tc(tm_q, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.lacc,
+                                 b.flag, b.plan.status, st));
   else
-    MOBA_TRY(moba::launch_fwd_attn(kq, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.flag, st));
+    MOBA_TRY(moba::launch_fwd_attn(kq, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.lacc, b.flag,
+                                   st));
   STAGE_END(MOBA_STAGE_FWD_ATTN);
   STAGE_BEGIN(MOBA_STAGE_FWD_FINALIZE);
-  MOBA_TRY(moba::launch_fwd_finalize(b.oacc, b.mref, b.flag, T * hq, d, static_cast<bf16*>(out), lse,
+  MOBA_TRY(moba::launch_fwd_finalize(b.oacc, b.lacc, b.mref, b.flag, T * hq, d, static_cast<bf16*>(out), lse,
                                      b.flag_list, st));
   MOBA_TRY(moba::launch_fwd_fallback(kq, kk, kv, plan, sel_idx, b.flag_list, hq, hkv, d, B, topk,
                                      static_cast<bf16*>(out), lse, st));

@@ -121,7 +121,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
              const bf16* __restrict__ cent_lo, const int32_t* __restrict__ cu,
              const int32_t* __restrict__ blk_off, const int32_t* __restrict__ tile_off, int batch,
              int nb_max, int h_q, int h_kv, int block_size, int topk, int32_t* __restrict__ sel_idx,
-             float* __restrict__ mref, int32_t* __restrict__ flag, float* __restrict__ oacc,
+             float* __restrict__ mref, int32_t* __restrict__ flag, float* __restrict__ oacc, float* __restrict__ lacc,
              int32_t* __restrict__ status) {
   using Ly = RouteLayout<D, NC, LISTN>;
   // Sift depth of a complete tree with LISTN - 1 nodes (children of the
@@ -188,13 +188,14 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   }
   if (nchunks > 0 && warp == 0) tc::tmem_alloc(sbase + Ly::HOLD_OFF, Ly::TMEM_COLS);
 
-  // Zero this tile's accumulator rows [O | l | pad] while the loads fly.
+  // Zero this tile's accumulator rows (O and l) while the loads fly.
   constexpr int OS = oacc_stride(D);
   for (int i = tid; i < nrows * (OS / 4); i += kThreads) {
     const int r = i / (OS / 4), c = i % (OS / 4);
     const size_t row = (size_t)(t0 + r) * h_q + h;
     reinterpret_cast<float4*>(oacc + row * OS)[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  if (tid < nrows) lacc[(size_t)(t0 + tid) * h_q + h] = 0.f;
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -405,7 +406,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
 template <int D, int NC, int LISTN>
 cudaError_t launch_route_t(const bf16* q, const bf16* k, const bf16* hi, const bf16* lo, const SeqPlan& p,
                            int h_q, int h_kv, int block_size, int topk, int32_t* sel, float* mref,
-                           int32_t* flag, float* oacc, int32_t* status, cudaStream_t st) {
+                           int32_t* flag, float* oacc, float* lacc, int32_t* status, cudaStream_t st) {
   const size_t smem = RouteLayout<D, NC, LISTN>::BYTES + 1024;
   auto kern = route_kernel<D, NC, LISTN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -414,7 +415,7 @@ cudaError_t launch_route_t(const bf16* q, const bf16* k, const bf16* hi, const b
   if (max_tiles == 0) return cudaSuccess;
   dim3 grid(max_tiles, h_q);
   kern<<<grid, kThreads, smem, st>>>(q, k, hi, lo, p.cu, p.blk_off, p.tile_off, p.batch, p.nb_max, h_q, h_kv,
-                                     block_size, topk, sel, mref, flag, oacc, status);
+                                     block_size, topk, sel, mref, flag, oacc, lacc, status);
   return cudaGetLastError();
 }
 
@@ -422,10 +423,10 @@ cudaError_t launch_route_t(const bf16* q, const bf16* k, const bf16* hi, const b
 
 cudaError_t launch_route(const bf16* q, const bf16* k, const bf16* hi, const bf16* lo, const SeqPlan& p,
                          int h_q, int h_kv, int d, int block_size, int topk, int32_t* sel, float* mref,
-                         int32_t* flag, float* oacc, int32_t* status, cudaStream_t st) {
+                         int32_t* flag, float* oacc, float* lacc, int32_t* status, cudaStream_t st) {
   const int k1 = topk - 1;
 #define MOBA_ROUTE(DD, NCC, LN) \
-  return launch_route_t<DD, NCC, LN>(q, k, hi, lo, p, h_q, h_kv, block_size, topk, sel, mref, flag, oacc, status, st)
+  return launch_route_t<DD, NCC, LN>(q, k, hi, lo, p, h_q, h_kv, block_size, topk, sel, mref, flag, oacc, lacc, status, st)
   if (d == 64) {
     if (k1 <= 32) MOBA_ROUTE(64, 32, 32);
     MOBA_ROUTE(64, 32, 64);
