@@ -34,9 +34,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem));
-}
 // Zero-fill variant: copies src_bytes (0 or 16) and zero-fills the rest.
 __device__ __forceinline__ void cp_async16_zfill(void* smem, const void* gmem, bool valid) {
   int n = valid ? 16 : 0;
@@ -74,23 +71,7 @@ __device__ __forceinline__ void red_add_v4(float* gaddr, float a, float b, float
                : "memory");
 }
 
-__device__ __forceinline__ void red_add_v2(float* gaddr, float a, float b) {
-  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};\n" ::"l"(gaddr), "f"(a), "f"(b) : "memory");
-}
 
-// Asynchronous bulk reduction (TMA engine): global[dst .. dst+bytes) +=
-// shared[src ..], fp32 elementwise; both 16-byte aligned, bytes % 16 == 0.
-__device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, const void* ssrc, uint32_t bytes) {
-  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(gdst),
-               "r"(smem_u32(ssrc)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Wait until this thread's bulk groups have finished reading shared memory.
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// Wait until this thread's bulk groups have fully completed.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;

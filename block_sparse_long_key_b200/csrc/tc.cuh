@@ -174,22 +174,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity, uint64
   }
 }
 
-// Named barrier `id` over `count` threads (a multiple of 32); id 0 is the
-// CTA-wide barrier.
-__device__ __forceinline__ void named_bar(uint32_t id, uint32_t count) {
-  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-// Same, returning the AND of `pred` over the participating threads.
-__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "barrier.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}\n"
-      : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(count) : "memory");
-  return r != 0;
-}
 // Registers `bytes` of expected async transactions with one arrival.
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t addr, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(bytes) : "memory");
@@ -207,11 +191,6 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int 
       " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(mbar)
       : "memory");
-}
-
-// One arrival on an mbarrier (release semantics at CTA scope).
-__device__ __forceinline__ void mbar_arrive(uint32_t addr) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(addr) : "memory");
 }
 
 }  // namespace tc
