@@ -57,10 +57,10 @@ cudaError_t launch_fwd_attn(const bf16* q, const bf16* k, const bf16* v, const S
                             int h_kv, int d, int block_size, float* oacc, float* lacc, int32_t* flag,
                             cudaStream_t st);
 
-// Tensor map over a [nrows, d] bf16 row table (16-byte aligned base) for
-// the tile::gather4 row gathers: 64-element boxes one row high, 128-byte
-// swizzle.
-cudaError_t make_row_map(CUtensorMap* map, const void* base, unsigned long long nrows, int d);
+// Tensor map over a [nrows, d] bf16 row table (16-byte aligned base):
+// 64-element boxes `box_rows` rows high, 128-byte swizzle (box_rows = 1 for
+// the tile::gather4 row gathers).
+cudaError_t make_row_map(CUtensorMap* map, const void* base, unsigned long long nrows, int d, int box_rows = 1);
 
 // tcgen05 forward attention for (d, B) = (64, 32), (128, 32), (128, 64);
 // `tm_q` is make_row_map over q as T*H_q rows.

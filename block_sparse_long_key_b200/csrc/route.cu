@@ -15,7 +15,7 @@
 // One CTA owns 128 consecutive queries of one sequence and one query head.
 // Their Q tile sits in tensor memory (thread t writes row t, the MMA's A
 // operand); a stream of centroid chunks (NC blocks each, double buffered,
-// cp.async into 128-byte-swizzled K-major shared memory) is the B operand of
+// TMA tile loads into 128-byte-swizzled K-major shared memory) is the B operand of
 // tcgen05.mma (M = 128 queries, N = NC blocks, bf16 in, fp32 accumulate into
 // tensor memory, double buffered): one thread issues q.c_hi + q.c_lo, which
 // carries ~16 mantissa bits of the fp32 centroid, while the CTA's 128 threads
@@ -60,8 +60,8 @@ struct RouteLayout {
   static constexpr uint32_t C_BUF = 2 * C_MAT;           // hi + lo
   static constexpr uint32_t HP_OFF = C_OFF + 2 * C_BUF;           // heap keys [LISTN][kThreads] u64
   static constexpr uint32_t BK_OFF = HP_OFF + LISTN * kThreads * 8;  // candidate keys [kBuf][kThreads] u64
-  static constexpr uint32_t MB_OFF = BK_OFF + kBuf * kThreads * 8;
-  static constexpr uint32_t HOLD_OFF = MB_OFF + 16;
+  static constexpr uint32_t MB_OFF = BK_OFF + kBuf * kThreads * 8;  // MMA done [2], chunk landed [2]
+  static constexpr uint32_t HOLD_OFF = MB_OFF + 32;
   static constexpr uint32_t BYTES = HOLD_OFF + 16;
   // Tensor memory: two NC-column score tiles, then Q (D bf16 = D/2 columns).
   static constexpr uint32_t TM_Q = 2 * NC;
@@ -117,8 +117,8 @@ __device__ __forceinline__ void warp_sort_desc(uint64_t (&x)[E], int lane) {
 
 template <int D, int NC, int LISTN>
 __global__ void __launch_bounds__(kThreads)
-route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ cent_hi,
-             const bf16* __restrict__ cent_lo, const int32_t* __restrict__ cu,
+route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __grid_constant__ CUtensorMap tm_hi,
+             const __grid_constant__ CUtensorMap tm_lo, const int32_t* __restrict__ cu,
              const int32_t* __restrict__ blk_off, const int32_t* __restrict__ tile_off, int batch,
              int nb_max, int h_q, int h_kv, int block_size, int topk, int32_t* __restrict__ sel_idx,
              float* __restrict__ mref, int32_t* __restrict__ flag, float* __restrict__ oacc, float* __restrict__ lacc,
@@ -132,7 +132,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   const uint32_t sbase = smem_u32(sm);
   uint64_t* heap = reinterpret_cast<uint64_t*>(sm + Ly::HP_OFF);
   uint64_t* bk = reinterpret_cast<uint64_t*>(sm + Ly::BK_OFF);
-  const uint32_t mbar0 = sbase + Ly::MB_OFF;
+  const uint32_t mbar0 = sbase + Ly::MB_OFF, mb_c0 = mbar0 + 16;
 
   const int ntiles = __ldg(tile_off + batch);
   const int tile = ntiles - 1 - (int)blockIdx.x;  // longest rows first
@@ -152,25 +152,22 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t qstride = (size_t)h_q * D;
 
-  // ---- loads: centroid chunks (hi, lo) into SW128 K-major layout
-  const size_t head0 = ((size_t)kvh * nb_max + cbase) * D;
+  // ---- loads: centroid chunks (hi, lo) into SW128 K-major layout by the
+  // TMA (thread 0): rows = global blocks of this KV head, boxes of NC rows x
+  // 64 values; rows past `nscan` (the next sequence's or head's blocks, or
+  // beyond the table: zero) are scored but never selected.
+  const int crow0 = kvh * nb_max + cbase;
   auto load_chunk = [&](int c, int buf) {
-    for (int i = tid; i < 2 * NC * (D / 8); i += kThreads) {
-      const int m = i / (NC * (D / 8));
-      const int rem = i % (NC * (D / 8));
-      const int n = rem / (D / 8), cc = rem % (D / 8);
-      const int jb = c * NC + n;
-      const bool ok = jb < nscan;
-      const size_t src = ok ? head0 + (size_t)jb * D + cc * 8 : 0;
-      unsigned char* dst = sm + Ly::C_OFF + buf * Ly::C_BUF + m * Ly::C_MAT + (cc >> 3) * Ly::C_REGION +
-                           tc::sw128_offset(n, cc & 7);
-      cp_async16_zfill(dst, (m ? cent_lo : cent_hi) + src, ok);
+    if (tid == 0) {
+      tc::mbar_arrive_expect_tx(mb_c0 + 8 * buf, 2 * Ly::C_MAT);
+#pragma unroll
+      for (int r = 0; r < Ly::KB; ++r) {
+        const uint32_t dst = sbase + Ly::C_OFF + buf * Ly::C_BUF + r * Ly::C_REGION;
+        tc::tma_load_2d(dst, &tm_hi, r * 64, crow0 + c * NC, mb_c0 + 8 * buf);
+        tc::tma_load_2d(dst + Ly::C_MAT, &tm_lo, r * 64, crow0 + c * NC, mb_c0 + 8 * buf);
+      }
     }
   };
-  if (nchunks > 0) load_chunk(0, 0);
-  cp_async_commit();
-  if (nchunks > 1) load_chunk(1, 1);
-  cp_async_commit();
 
   // ---- per-thread selection state; TMEM + barriers
   const bool row_ok = tid < nrows;
@@ -184,6 +181,8 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   if (tid == 0) {
     tc::mbar_init(mbar0, 1);
     tc::mbar_init(mbar0 + 8, 1);
+    tc::mbar_init(mb_c0, 1);
+    tc::mbar_init(mb_c0 + 8, 1);
     tc::mbar_init_fence();
   }
   if (nchunks > 0 && warp == 0) tc::tmem_alloc(sbase + Ly::HOLD_OFF, Ly::TMEM_COLS);
@@ -199,6 +198,8 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  if (nchunks > 0) load_chunk(0, 0);
+  if (nchunks > 1) load_chunk(1, 1);
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
   constexpr uint32_t idesc = tc::idesc_bf16_f32(kTM, NC);
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -285,10 +286,14 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
   bool ok = true;
   for (int c = 0; c < nchunks && ok; ++c) {
     const int buf = c & 1;
-    if (c == 0 && nchunks > 1) cp_async_wait<1>(); else cp_async_wait<0>();
-    tc::fence_proxy_async();
-    tc::fence_before_sync();
-    __syncthreads();
+    {
+      const bool landed = tc::mbar_wait(mb_c0 + 8 * buf, (c >> 1) & 1);
+      tc::fence_before_sync();
+      if (!__syncthreads_and(landed)) {
+        ok = false;
+        break;
+      }
+    }
     if (tid == 0) {
       tc::fence_after_sync();
       const uint32_t d_tmem = tmem + (uint32_t)(buf * NC);
@@ -315,7 +320,6 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
         break;
       }
       if (c + 1 < nchunks) load_chunk(c + 1, (c + 1) & 1);
-      cp_async_commit();
       tc::fence_after_sync();
       select_chunk(pc, pc & 1);
       tc::fence_before_sync();
@@ -332,14 +336,16 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16*
       ok = false;
     }
   }
-  cp_async_wait<0>();
   tc::fence_before_sync();
   __syncthreads();
   if (!ok) {
-    // A tensor-core completion never arrived: record it, give the MMAs in
-    // flight a bounded chance to drain, release TMEM, leave outputs unwritten.
+    // A wait gave up: record it, give the MMAs and chunk loads in flight a
+    // bounded chance to drain (a wait on a phase that is not pending returns
+    // at once), release TMEM, leave outputs unwritten.
     if (tid == 0) set_status(status, kStatusTimeout);
     tc::mbar_wait(mbar0 + 8 * ((nchunks - 1) & 1), ((nchunks - 1) >> 1) & 1, 100000000ull);
+    for (int b2 = 0; b2 < 2; ++b2)
+      for (int ph = 0; ph < 2; ++ph) tc::mbar_wait(mb_c0 + 8 * b2, ph, 20000000ull);
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, Ly::TMEM_COLS);
     return;
@@ -412,10 +418,16 @@ cudaError_t launch_route_t(const bf16* q, const bf16* k, const bf16* hi, const b
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int max_tiles = p.total_tokens / kTM + p.batch;
-  if (max_tiles == 0) return cudaSuccess;
+  if (max_tiles == 0 || p.nb_max == 0) return cudaSuccess;
+  CUtensorMap tm_hi, tm_lo;  // the centroid tables as h_kv * nb_max rows of D
+  const unsigned long long nrows = (unsigned long long)h_kv * p.nb_max;
+  e = make_row_map(&tm_hi, hi, nrows, D, NC);
+  if (e != cudaSuccess) return e;
+  e = make_row_map(&tm_lo, lo, nrows, D, NC);
+  if (e != cudaSuccess) return e;
   dim3 grid(max_tiles, h_q);
-  kern<<<grid, kThreads, smem, st>>>(q, k, hi, lo, p.cu, p.blk_off, p.tile_off, p.batch, p.nb_max, h_q, h_kv,
-                                     block_size, topk, sel, mref, flag, oacc, lacc, status);
+  kern<<<grid, kThreads, smem, st>>>(q, k, tm_hi, tm_lo, p.cu, p.blk_off, p.tile_off, p.batch, p.nb_max, h_q,
+                                     h_kv, block_size, topk, sel, mref, flag, oacc, lacc, status);
   return cudaGetLastError();
 }
 

@@ -179,6 +179,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t addr, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(bytes) : "memory");
 }
 
+// TMA 2-D tile load: the box at (x, y) of `tmap` into shared memory at
+// `dst` (128-byte aligned; a 1024-byte aligned tile gets the SW128 layout),
+// completion counted in bytes on `mbar`.  No cluster multicast.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y, uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(mbar)
+      : "memory");
+}
+
 // TMA row gather: rows r0..r3 of a 2-D tensor map (box: 64 elements x one
 // row, 128-byte swizzle), columns c0 .. c0+63, into 4 consecutive 128-byte
 // rows of shared memory at `dst` (128-byte aligned; the swizzle follows the

@@ -1,6 +1,7 @@
-// Host side of the TMA row gathers: tensor maps over [rows, d] bf16 tables
-// (Q or dO viewed as T*H_q rows of d values), 64-element (128-byte) boxes
-// one row high with the 128-byte swizzle, as the tile::gather4 loads need.
+// Host side of the TMA loads: tensor maps over [rows, d] bf16 tables (Q or
+// dO viewed as T*H_q rows of d values, or the block centroids), boxes of 64
+// elements (128 bytes) by `box_rows` rows with the 128-byte swizzle (one row
+// high for the tile::gather4 row gathers).
 // The driver entry point is looked up once through the runtime.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -31,13 +32,14 @@ EncodeTiled encode_fn() {
 
 }  // namespace
 
-cudaError_t make_row_map(CUtensorMap* map, const void* base, unsigned long long nrows, int d) {
+cudaError_t make_row_map(CUtensorMap* map, const void* base, unsigned long long nrows, int d, int box_rows) {
   EncodeTiled fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || nrows == 0) return cudaErrorInvalidValue;
   const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)nrows};
   const cuuint64_t strides[1] = {(cuuint64_t)d * 2};  // bytes between rows
-  const cuuint32_t box[2] = {64, 1};
+  if (box_rows < 1 || box_rows > 256) return cudaErrorInvalidValue;
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
