@@ -56,15 +56,15 @@ __global__ void __launch_bounds__(BwdCfg<D, BLK>::NT)
 bwd_attn_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                 const bf16* __restrict__ dout, const float* __restrict__ lse, const float* __restrict__ dsum,
                 const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch, int nb_max,
-                int h_q, int h_kv, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
+                int h_q, int h_kv, int lead, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
                 float* __restrict__ dqacc, bf16* __restrict__ dk, bf16* __restrict__ dv) {
   using C = BwdCfg<D, BLK>;
   constexpr int TR = C::TR, KG = C::KG, NW = C::NW, NT = C::NT;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   BwdSmem<D, BLK>& sm = *reinterpret_cast<BwdSmem<D, BLK>*>(smem_raw);
 
-  const int gb = blockIdx.x;
-  const int kvh = blockIdx.y;
+  const BucketOrder bo = bucket_order(blockIdx.x, nb_max, h_kv, lead);
+  const int gb = bo.gb, kvh = bo.kvh;
   if (gb >= __ldg(blk_off + batch)) return;
   const int bucket = kvh * nb_max + gb;
   const int beg = __ldg(ptr + bucket), end = __ldg(ptr + bucket + 1);
@@ -348,9 +348,10 @@ cudaError_t launch_bwd_t(const bf16* q, const bf16* k, const bf16* v, const bf16
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (p.nb_max == 0) return cudaSuccess;
-  dim3 grid(p.nb_max, h_kv);
+  dim3 grid(p.nb_max * h_kv);
+  const int lead = bucket_lead((long long)p.total_tokens * (h_q / h_kv), D * 4);
   kern<<<grid, BwdCfg<D, BLK>::NT, smem, st>>>(q, k, v, dout, lse, dsum, p.cu, p.blk_off, p.batch, p.nb_max, h_q,
-                                               h_kv, ptr, rows, dqacc, dk, dv);
+                                               h_kv, lead, ptr, rows, dqacc, dk, dv);
   return cudaGetLastError();
 }
 

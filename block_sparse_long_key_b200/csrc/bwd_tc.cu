@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kThreads)
 bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__ k, const bf16* __restrict__ v,
               const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ lse, const float* __restrict__ dsum,
               const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch, int nb_max,
-              int h_q, int h_kv, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
+              int h_q, int h_kv, int lead, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
               float* __restrict__ dqacc, bf16* __restrict__ dk, bf16* __restrict__ dv,
               int32_t* __restrict__ status) {
   using Ly = BwdTcLayout<D, BLK>;
@@ -91,8 +91,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
   const uint32_t sbase = smem_u32(sm);
   const uint32_t mb_s = sbase + Ly::MB_OFF, mb_g = mb_s + 8, mb_q = mb_s + 16;
 
-  const int gb = blockIdx.x;
-  const int kvh = blockIdx.y;
+  const BucketOrder bo = bucket_order(blockIdx.x, nb_max, h_kv, lead);
+  const int gb = bo.gb, kvh = bo.kvh;
   if (gb >= __ldg(blk_off + batch)) return;
   const int bucket = kvh * nb_max + gb;
   const int beg = __ldg(ptr + bucket), end = __ldg(ptr + bucket + 1);
@@ -365,8 +365,10 @@ cudaError_t launch_bwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v,
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);     \
     if (e != cudaSuccess) return e;                                                                          \
     if (p.nb_max == 0) return cudaSuccess;                                                                   \
-    kern<<<dim3(p.nb_max, h_kv), kThreads, smem, st>>>(tm_q, k, v, tm_do, lse, dsum, p.cu, p.blk_off, p.batch, \
-                                                       p.nb_max, h_q, h_kv, ptr, rows, dqacc, dk, dv, status); \
+    const int lead = bucket_lead((long long)p.total_tokens * (h_q / h_kv), DD * 4);                          \
+    kern<<<dim3(p.nb_max * h_kv), kThreads, smem, st>>>(tm_q, k, v, tm_do, lse, dsum, p.cu, p.blk_off, p.batch, \
+                                                       p.nb_max, h_q, h_kv, lead, ptr, rows, dqacc, dk, dv,   \
+                                                       status);                                                \
     return cudaGetLastError();                                                                               \
   } while (0)
   if (d == 64 && block_size == 32) MOBA_BWD_TC(64, 32);

@@ -30,6 +30,42 @@ __device__ __forceinline__ int upper_seq(const int32_t* off, int n, int x) {
   return lo;
 }
 
+// Dispatch order of the attention kernels' CTAs, one per (key block, KV
+// head), over a one-dimensional grid of nb_max * h_kv.  A block is a
+// candidate for every later query, so a head's buckets shrink with the block
+// index and its first blocks are its longest CTAs.  CTAs go head by head,
+// which keeps the accumulator rows of the heads in flight resident in L2,
+// except that the first nb_max / 8 blocks of head h are issued beside the
+// short CTAs of head h - lead: long CTAs start `lead` head-windows early
+// instead of trailing the grid on the last head.  lead = 0 is plain head-major
+// order (for heads whose accumulator alone fills L2; see bucket_lead()).
+struct BucketOrder {
+  int gb, kvh;
+};
+__device__ __forceinline__ BucketOrder bucket_order(int L, int nb_max, int h_kv, int lead) {
+  lead = lead < h_kv ? lead : h_kv;
+  const int big = nb_max / 8 > 1 ? nb_max / 8 : 1;
+  const int small = nb_max - big;
+  BucketOrder o;
+  if (L < lead * big) {  // the first heads' long CTAs
+    o.kvh = L / big;
+    o.gb = L % big;
+    return o;
+  }
+  L -= lead * big;
+  const int mid = (h_kv - lead) * nb_max;
+  if (L < mid) {  // window s: long CTAs of head s + lead, then short ones of head s
+    const int s = L / nb_max, r = L % nb_max;
+    o.kvh = r < big ? s + lead : s;
+    o.gb = r;
+    return o;
+  }
+  L -= mid;  // the last heads' short CTAs (small > 0 whenever this is reached)
+  o.kvh = h_kv - lead + L / small;
+  o.gb = big + L % small;
+  return o;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

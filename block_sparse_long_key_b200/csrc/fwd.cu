@@ -59,7 +59,7 @@ template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads)
 fwd_attn_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                 const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch, int nb_max,
-                int h_q, int h_kv, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
+                int h_q, int h_kv, int lead, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
                 const float* __restrict__ mref, float* __restrict__ oacc, float* __restrict__ lacc,
                 int32_t* __restrict__ flag) {
   constexpr int KC = BLK < 64 ? BLK : 64;  // keys per register chunk
@@ -68,8 +68,8 @@ fwd_attn_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
   extern __shared__ __align__(128) unsigned char smem_raw[];
   FwdSmem<D, BLK>& sm = *reinterpret_cast<FwdSmem<D, BLK>*>(smem_raw);
 
-  const int gb = blockIdx.x;
-  const int kvh = blockIdx.y;
+  const BucketOrder bo = bucket_order(blockIdx.x, nb_max, h_kv, lead);
+  const int gb = bo.gb, kvh = bo.kvh;
   if (gb >= __ldg(blk_off + batch)) return;
   const int bucket = kvh * nb_max + gb;
   const int beg = __ldg(ptr + bucket), end = __ldg(ptr + bucket + 1);
@@ -339,8 +339,9 @@ cudaError_t launch_fwd_t(const bf16* q, const bf16* k, const bf16* v, const SeqP
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (p.nb_max == 0) return cudaSuccess;
-  dim3 grid(p.nb_max, h_kv);
-  kern<<<grid, kThreads, smem, st>>>(q, k, v, p.cu, p.blk_off, p.batch, p.nb_max, h_q, h_kv, ptr, rows, mref,
+  dim3 grid(p.nb_max * h_kv);
+  const int lead = bucket_lead((long long)p.total_tokens * (h_q / h_kv), D * 4 + 4);
+  kern<<<grid, kThreads, smem, st>>>(q, k, v, p.cu, p.blk_off, p.batch, p.nb_max, h_q, h_kv, lead, ptr, rows, mref,
                                      oacc, lacc, flag);
   return cudaGetLastError();
 }

@@ -33,11 +33,21 @@ cudaError_t launch_conv_centroid(const bf16* k, const float* conv_w, int conv_wi
                                  int h_kv, int d, int block_size, bf16* k_out, float* cent,
                                  bf16* cent_hi, bf16* cent_lo, cudaStream_t st);
 
-// Forward accumulator rows: O (d floats), l, 3 floats of padding.
 // Forward accumulator: rows of d floats (the unnormalised O, 256- or
 // 512-byte rows, so each starts on an L2 line) and, separately, one float l
 // per row.
 __host__ __device__ constexpr int oacc_stride(int d) { return d; }
+
+// How many head-windows early the attention kernels issue a head's longest
+// CTAs (bucket_order): as many as let those heads' accumulator rows share
+// half of L2 with the current head's, at most 2; 0 when one head's rows
+// already fill that much.
+inline int bucket_lead(long long rows_per_kv_head, int row_bytes) {
+  const long long head = rows_per_kv_head * row_bytes;
+  if (head <= 0) return 0;
+  const long long n = (64ll << 20) / head - 1;
+  return (int)(n < 0 ? 0 : (n > 2 ? 2 : n));
+}
 
 cudaError_t launch_route(const bf16* q, const bf16* k, const bf16* cent_hi, const bf16* cent_lo,
                          const SeqPlan& p, int h_q, int h_kv, int d, int block_size, int topk,

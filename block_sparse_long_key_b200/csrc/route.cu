@@ -135,9 +135,11 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   const uint32_t mbar0 = sbase + Ly::MB_OFF, mb_c0 = mbar0 + 16;
 
   const int ntiles = __ldg(tile_off + batch);
-  const int tile = ntiles - 1 - (int)blockIdx.x;  // longest rows first
+  // Longest rows first, every head's together: a CTA's time grows with its
+  // rows' position, so the grid ends on short tiles.
+  const int h = (int)(blockIdx.x % (unsigned)h_q);
+  const int tile = ntiles - 1 - (int)(blockIdx.x / (unsigned)h_q);
   if (tile < 0) return;
-  const int h = blockIdx.y;
   const int kvh = h / (h_q / h_kv);
   const int s = upper_seq(tile_off, batch, tile);
   const int seq0 = __ldg(cu + s);
@@ -425,7 +427,7 @@ cudaError_t launch_route_t(const bf16* q, const bf16* k, const bf16* hi, const b
   if (e != cudaSuccess) return e;
   e = make_row_map(&tm_lo, lo, nrows, D, NC);
   if (e != cudaSuccess) return e;
-  dim3 grid(max_tiles, h_q);
+  dim3 grid(max_tiles * h_q);
   kern<<<grid, kThreads, smem, st>>>(q, k, tm_hi, tm_lo, p.cu, p.blk_off, p.tile_off, p.batch, p.nb_max, h_q,
                                      h_kv, block_size, topk, sel, mref, flag, oacc, lacc, status);
   return cudaGetLastError();
