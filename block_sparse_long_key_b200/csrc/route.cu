@@ -17,10 +17,12 @@
 // operand); a stream of centroid chunks (NC blocks each, double buffered,
 // TMA tile loads into 128-byte-swizzled K-major shared memory) is the B operand of
 // tcgen05.mma (M = 128 queries, N = NC blocks, bf16 in, fp32 accumulate into
-// tensor memory, double buffered): one thread issues q.c_hi + q.c_lo, which
-// carries ~16 mantissa bits of the fp32 centroid, while the CTA's 128 threads
-// select on the previous chunk.  Thread t owns query row t, which is TMEM lane
-// t: tcgen05.ld hands it that row's NC scores in registers.  Scores above the
+// tensor memory, three score tiles at d = 64, two at d = 128): a producer
+// warp issues the loads and q.c_hi + q.c_lo, which carries ~16 mantissa bits
+// of the fp32 centroid, while the four selecting warps work on earlier chunks
+// (mbarrier hand-offs per score tile, no block-wide barrier per chunk).
+// Thread t owns query row t, which is TMEM lane t: tcgen05.ld hands it that
+// row's NC scores in registers.  Scores above the
 // thread's running threshold (the worst of its current k-1 best) go to a
 // small per-thread candidate buffer in shared memory; the whole warp flushes
 // the buffers together.  The k-1 kept entries form a binary min-heap of
@@ -42,7 +44,8 @@ namespace moba {
 namespace {
 
 constexpr int kTM = kRouteTile;  // query rows per CTA (= TMEM lanes)
-constexpr int kThreads = 128;
+constexpr int kSel = 128;        // selecting threads: thread t owns row t (warps 0-3)
+constexpr int kThreads = kSel + 32;  // + one producer warp (chunk loads, MMAs)
 constexpr uint64_t kKeyMax = ~0ull;  // heap padding: never the minimum
 // An empty live slot: the key of score -inf (below every finite score), so
 // the root's score reads back as -inf until k-1 blocks have been admitted.
@@ -52,19 +55,22 @@ constexpr int kGroup = 4;  // columns appended between buffer checks
 
 template <int D, int NC, int LISTN>
 struct RouteLayout {
+  static constexpr int NB = D == 64 ? 3 : 2;              // score tiles in tensor memory
   static constexpr int kBuf = 6;                          // candidate buffer slots per thread
   static constexpr int KB = D / 64;                       // 128-byte K blocks
   static constexpr uint32_t C_OFF = 0;
   static constexpr uint32_t C_REGION = NC * 128;
   static constexpr uint32_t C_MAT = KB * C_REGION;       // hi or lo of one chunk
   static constexpr uint32_t C_BUF = 2 * C_MAT;           // hi + lo
-  static constexpr uint32_t HP_OFF = C_OFF + 2 * C_BUF;           // heap keys [LISTN][kThreads] u64
-  static constexpr uint32_t BK_OFF = HP_OFF + LISTN * kThreads * 8;  // candidate keys [kBuf][kThreads] u64
-  static constexpr uint32_t MB_OFF = BK_OFF + kBuf * kThreads * 8;  // MMA done [2], chunk landed [2]
-  static constexpr uint32_t HOLD_OFF = MB_OFF + 32;
+  static constexpr uint32_t HP_OFF = C_OFF + 2 * C_BUF;           // heap keys [LISTN][kSel] u64
+  static constexpr uint32_t BK_OFF = HP_OFF + LISTN * kSel * 8;  // candidate keys [kBuf][kSel] u64
+  // mbarriers: score tile full [NB] (MMA done), score tile empty [NB] (read
+  // by the four selecting warps), chunk landed [2], Q in tensor memory.
+  static constexpr uint32_t MB_OFF = BK_OFF + kBuf * kSel * 8;
+  static constexpr uint32_t HOLD_OFF = MB_OFF + 8 * (2 * NB + 3);
   static constexpr uint32_t BYTES = HOLD_OFF + 16;
-  // Tensor memory: two NC-column score tiles, then Q (D bf16 = D/2 columns).
-  static constexpr uint32_t TM_Q = 2 * NC;
+  // Tensor memory: NB NC-column score tiles, then Q (D bf16 = D/2 columns).
+  static constexpr uint32_t TM_Q = NB * NC;
   static constexpr uint32_t TMEM_COLS = 128;
   static_assert((LISTN & (LISTN - 1)) == 0, "heap is a complete tree of LISTN - 1 nodes");
   static_assert(C_REGION % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
@@ -116,7 +122,7 @@ __device__ __forceinline__ void warp_sort_desc(uint64_t (&x)[E], int lane) {
 }
 
 template <int D, int NC, int LISTN>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)
 route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __grid_constant__ CUtensorMap tm_hi,
              const __grid_constant__ CUtensorMap tm_lo, const int32_t* __restrict__ cu,
              const int32_t* __restrict__ blk_off, const int32_t* __restrict__ tile_off, int batch,
@@ -132,7 +138,8 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   const uint32_t sbase = smem_u32(sm);
   uint64_t* heap = reinterpret_cast<uint64_t*>(sm + Ly::HP_OFF);
   uint64_t* bk = reinterpret_cast<uint64_t*>(sm + Ly::BK_OFF);
-  const uint32_t mbar0 = sbase + Ly::MB_OFF, mb_c0 = mbar0 + 16;
+  const uint32_t mb_full = sbase + Ly::MB_OFF, mb_empty = mb_full + 8 * Ly::NB;
+  const uint32_t mb_c0 = mb_empty + 8 * Ly::NB, mb_q = mb_c0 + 16;
 
   const int ntiles = __ldg(tile_off + batch);
   // Longest rows first, every head's together: a CTA's time grows with its
@@ -155,36 +162,39 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   const size_t qstride = (size_t)h_q * D;
 
   // ---- loads: centroid chunks (hi, lo) into SW128 K-major layout by the
-  // TMA (thread 0): rows = global blocks of this KV head, boxes of NC rows x
-  // 64 values; rows past `nscan` (the next sequence's or head's blocks, or
-  // beyond the table: zero) are scored but never selected.
+  // TMA (the producer thread): rows = global blocks of this KV head, boxes of
+  // NC rows x 64 values; rows past `nscan` (the next sequence's or head's
+  // blocks, or beyond the table: zero) are scored but never selected.
   const int crow0 = kvh * nb_max + cbase;
   auto load_chunk = [&](int c, int buf) {
-    if (tid == 0) {
-      tc::mbar_arrive_expect_tx(mb_c0 + 8 * buf, 2 * Ly::C_MAT);
+    tc::mbar_arrive_expect_tx(mb_c0 + 8 * buf, 2 * Ly::C_MAT);
 #pragma unroll
-      for (int r = 0; r < Ly::KB; ++r) {
-        const uint32_t dst = sbase + Ly::C_OFF + buf * Ly::C_BUF + r * Ly::C_REGION;
-        tc::tma_load_2d(dst, &tm_hi, r * 64, crow0 + c * NC, mb_c0 + 8 * buf);
-        tc::tma_load_2d(dst + Ly::C_MAT, &tm_lo, r * 64, crow0 + c * NC, mb_c0 + 8 * buf);
-      }
+    for (int r = 0; r < Ly::KB; ++r) {
+      const uint32_t dst = sbase + Ly::C_OFF + buf * Ly::C_BUF + r * Ly::C_REGION;
+      tc::tma_load_2d(dst, &tm_hi, r * 64, crow0 + c * NC, mb_c0 + 8 * buf);
+      tc::tma_load_2d(dst + Ly::C_MAT, &tm_lo, r * 64, crow0 + c * NC, mb_c0 + 8 * buf);
     }
   };
 
   // ---- per-thread selection state; TMEM + barriers
+  const bool sel_thread = tid < kSel;
   const bool row_ok = tid < nrows;
   const int my_b = row_ok ? (p0 + tid) / block_size : 0;
   // Min-heap of the kept keys: k1 live slots start empty (score -inf),
   // padding slots up to LISTN-1 hold kKeyMax and never surface.
-  for (int sl = 0; sl < LISTN; ++sl) heap[sl * kThreads + tid] = sl < k1 ? kKeyEmpty : kKeyMax;
+  if (sel_thread)
+    for (int sl = 0; sl < LISTN; ++sl) heap[sl * kSel + tid] = sl < k1 ? kKeyEmpty : kKeyMax;
   uint64_t root_key = kKeyEmpty;  // the heap's root: the worst kept key
   float tau = -INFINITY;          // its score
   int cnt = 0;                    // buffered candidate keys
   if (tid == 0) {
-    tc::mbar_init(mbar0, 1);
-    tc::mbar_init(mbar0 + 8, 1);
+    for (int i = 0; i < Ly::NB; ++i) {
+      tc::mbar_init(mb_full + 8 * i, 1);
+      tc::mbar_init(mb_empty + 8 * i, kSel / 32);
+    }
     tc::mbar_init(mb_c0, 1);
     tc::mbar_init(mb_c0 + 8, 1);
+    tc::mbar_init(mb_q, kSel / 32);
     tc::mbar_init_fence();
   }
   if (nchunks > 0 && warp == 0) tc::tmem_alloc(sbase + Ly::HOLD_OFF, Ly::TMEM_COLS);
@@ -200,12 +210,13 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  if (nchunks > 0) load_chunk(0, 0);
-  if (nchunks > 1) load_chunk(1, 1);
+  const bool producer = tid == kSel;  // lane 0 of the last warp
+  if (producer && nchunks > 0) load_chunk(0, 0);
+  if (producer && nchunks > 1) load_chunk(1, 1);
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
   constexpr uint32_t idesc = tc::idesc_bf16_f32(kTM, NC);
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  if (nchunks > 0) {
+  if (nchunks > 0 && sel_thread) {
     // Q row `tid` -> TMEM lane `tid`, columns TM_Q .. TM_Q + D/2 (bf16 pairs).
     const bf16* qrow = q + (size_t)(t0 + tid) * qstride + (size_t)h * D;
 #pragma unroll
@@ -222,6 +233,9 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
       tc::tmem_st32(tmem + lane_base + Ly::TM_Q + half * 32, w);
     }
     tc::tmem_st_wait();
+    tc::fence_before_sync();
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(mb_q);
   }
 
   // Admit a key above the root: replace the root and sift it down.
@@ -232,19 +246,19 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
 #pragma unroll
     for (int lvl = 0; lvl < kHeapDepth; ++lvl) {
       const int c1 = 2 * pos + 1;
-      const uint64_t k1v = heap[c1 * kThreads + tid];
-      const uint64_t k2v = heap[(c1 + 1) * kThreads + tid];
+      const uint64_t k1v = heap[c1 * kSel + tid];
+      const uint64_t k2v = heap[(c1 + 1) * kSel + tid];
       const bool left = k1v < k2v;
       const uint64_t km = left ? k1v : k2v;
       if (!done && km < key) {
-        heap[pos * kThreads + tid] = km;
+        heap[pos * kSel + tid] = km;
         if (lvl == 0) root = km;
         pos = left ? c1 : c1 + 1;
       } else {
         done = true;
       }
     }
-    heap[pos * kThreads + tid] = key;
+    heap[pos * kSel + tid] = key;
     root_key = root;
     tau = from_order_bits((uint32_t)(root >> 32));
   };
@@ -255,18 +269,14 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   auto flush_round = [&]() {
     if (cnt > 0) {
       --cnt;
-      const uint64_t key = bk[cnt * kThreads + tid];
+      const uint64_t key = bk[cnt * kSel + tid];
       if (key > root_key) admit(key);
     }
   };
 
-  auto select_chunk = [&](int c, int buf) {
-    uint32_t v[NC];
-    const uint32_t taddr = tmem + lane_base + (uint32_t)(buf * NC);
-#pragma unroll
-    for (int hf = 0; hf < NC / 32; ++hf)
-      tc::tmem_ld32(taddr + hf * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[hf * 32]));
-    tc::tmem_ld_wait();
+  // Selection on one chunk's scores: those above the row's threshold go to
+  // the candidate buffer, which the warp flushes into the heaps in rounds.
+  auto select_scores = [&](const uint32_t (&v)[NC], int c) {
     const int jbase = c * NC;
 #pragma unroll
     for (int g = 0; g < NC / kGroup; ++g) {
@@ -278,27 +288,33 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
         const int j = jbase + col;
         // Blocks arrive in ascending j, so a score equal to tau (the root's,
         // which has a lower index) never wins: the strict test is exact.
-        if (j < my_b && x > tau) bk[(cnt++) * kThreads + tid] = make_key(x, j);
+        if (j < my_b && x > tau) bk[(cnt++) * kSel + tid] = make_key(x, j);
       }
     }
   };
 
-  // All waits are decided block-wide (__syncthreads_and), so every thread
-  // takes the same path if a tensor-core completion never arrives.
+  // Producer (one thread): chunk c's MMAs go into score tile c % NB once the
+  // chunk has landed and the four selecting warps have read the tile's
+  // previous contents; the load of chunk c + 1 reuses the shared-memory
+  // buffer of chunk c - 1 once that chunk's MMAs are done.  Selecting warps:
+  // wait for tile c % NB, read it into registers, release it, select.  No
+  // block-wide barrier inside the loop, so the warps drift apart by up to NB
+  // chunks.  Every wait is bounded and decided warp-wide; one that gives up
+  // ends the loop, and the block agrees on the outcome afterwards.
   bool ok = true;
-  for (int c = 0; c < nchunks && ok; ++c) {
-    const int buf = c & 1;
-    {
-      const bool landed = tc::mbar_wait(mb_c0 + 8 * buf, (c >> 1) & 1);
-      tc::fence_before_sync();
-      if (!__syncthreads_and(landed)) {
-        ok = false;
-        break;
+  if (producer && nchunks > 0) {
+    ok = tc::mbar_wait(mb_q, 0);
+    for (int c = 0; c < nchunks && ok; ++c) {
+      const int buf = c & 1, sc = c % Ly::NB;
+      if (c >= 1 && c + 1 < nchunks) {
+        const int pc = c - 1;
+        if (!(ok = tc::mbar_wait(mb_full + 8 * (pc % Ly::NB), (pc / Ly::NB) & 1))) break;
+        load_chunk(c + 1, (c + 1) & 1);
       }
-    }
-    if (tid == 0) {
+      if (!(ok = tc::mbar_wait(mb_c0 + 8 * buf, (c >> 1) & 1))) break;
+      if (c >= Ly::NB && !(ok = tc::mbar_wait(mb_empty + 8 * sc, ((c / Ly::NB) - 1) & 1))) break;
       tc::fence_after_sync();
-      const uint32_t d_tmem = tmem + (uint32_t)(buf * NC);
+      const uint32_t d_tmem = tmem + (uint32_t)(sc * NC);
       const uint32_t qa = tmem + Ly::TM_Q;  // lane 0, Q columns
       const uint32_t ca = sbase + Ly::C_OFF + buf * Ly::C_BUF;
 #pragma unroll
@@ -312,44 +328,46 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
         tc::mma_bf16_ts(d_tmem, qa + kk * 8, tc::sw128_desc(ca + Ly::C_MAT + (kk >> 2) * Ly::C_REGION + koff), idesc,
                         1u);
       }
-      tc::mma_commit(mbar0 + 8 * buf);
+      tc::mma_commit(mb_full + 8 * sc);
     }
-    if (c >= 1) {
-      const int pc = c - 1;
-      const bool got = tc::mbar_wait(mbar0 + 8 * (pc & 1), (pc >> 1) & 1);
-      if (!__syncthreads_and(got)) {
+  } else if (sel_thread) {
+    for (int c = 0; c < nchunks; ++c) {
+      const int sc = c % Ly::NB;
+      const bool got = tc::mbar_wait(mb_full + 8 * sc, (c / Ly::NB) & 1);
+      if (!__all_sync(kFull, got)) {
         ok = false;
         break;
       }
-      if (c + 1 < nchunks) load_chunk(c + 1, (c + 1) & 1);
       tc::fence_after_sync();
-      select_chunk(pc, pc & 1);
+      uint32_t v[NC];
+      const uint32_t taddr = tmem + lane_base + (uint32_t)(sc * NC);
+#pragma unroll
+      for (int hf = 0; hf < NC / 32; ++hf)
+        tc::tmem_ld32(taddr + hf * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[hf * 32]));
+      tc::tmem_ld_wait();
       tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(mb_empty + 8 * sc);
+      select_scores(v, c);
     }
-  }
-  if (nchunks > 0 && ok) {
-    const int pc = nchunks - 1;
-    const bool got = tc::mbar_wait(mbar0 + 8 * (pc & 1), (pc >> 1) & 1);
-    if (__syncthreads_and(got)) {
-      tc::fence_after_sync();
-      select_chunk(pc, pc & 1);
+    if (ok)
       while (__any_sync(kFull, cnt > 0)) flush_round();
-    } else {
-      ok = false;
-    }
   }
   tc::fence_before_sync();
-  __syncthreads();
+  ok = __syncthreads_and(ok);
   if (!ok) {
     // A wait gave up: record it, give the MMAs and chunk loads in flight a
     // bounded chance to drain (a wait on a phase that is not pending returns
     // at once), release TMEM, leave outputs unwritten.
     if (tid == 0) set_status(status, kStatusTimeout);
-    tc::mbar_wait(mbar0 + 8 * ((nchunks - 1) & 1), ((nchunks - 1) >> 1) & 1, 100000000ull);
-    for (int b2 = 0; b2 < 2; ++b2)
-      for (int ph = 0; ph < 2; ++ph) tc::mbar_wait(mb_c0 + 8 * b2, ph, 20000000ull);
+    if (producer) {
+      for (int i = 0; i < Ly::NB; ++i)
+        for (int ph = 0; ph < 2; ++ph) tc::mbar_wait(mb_full + 8 * i, ph, 20000000ull);
+      for (int b2 = 0; b2 < 2; ++b2)
+        for (int ph = 0; ph < 2; ++ph) tc::mbar_wait(mb_c0 + 8 * b2, ph, 20000000ull);
+    }
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, Ly::TMEM_COLS);
+    if (nchunks > 0 && warp == 0) tc::tmem_dealloc(tmem, Ly::TMEM_COLS);
     return;
   }
   if (nchunks > 0 && warp == 0) {
@@ -370,7 +388,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const int i = lane * E + e;
-      const uint64_t key = i < k1 ? heap[i * kThreads + rr] : kKeyEmpty;
+      const uint64_t key = i < k1 ? heap[i * kSel + rr] : kKeyEmpty;
       const bool real = key != kKeyEmpty;
       kept_n += __popc(__ballot_sync(kFull, real));
       y[e] = real ? (key & 0xffffffffull) : 0ull;  // inverted index: larger = lower block
