@@ -89,36 +89,24 @@ __device__ __forceinline__ uint64_t make_key(float x, int j) {
   return ((uint64_t)order_bits(x) << 32) | (uint64_t)(0xffffffffu - (uint32_t)j);
 }
 
-// One compare-exchange step of a bitonic network over the 32E keys a warp
-// holds (key i = lane * E + e): key i is paired with key i ^ j, and a block
-// of k keys is ordered descending where (i & k) == 0, ascending elsewhere.
-template <int E>
-__device__ __forceinline__ void bitonic_step(uint64_t (&x)[E], int lane, int k, int j) {
-  if (j < E) {  // E == 2, j == 1: both keys of the lane, same block direction
-    const bool desc = ((lane * E) & k) == 0;
-    const uint64_t hi = x[0] > x[E - 1] ? x[0] : x[E - 1];
-    const uint64_t lo = x[0] > x[E - 1] ? x[E - 1] : x[0];
-    x[0] = desc ? hi : lo;
-    x[E - 1] = desc ? lo : hi;
-  } else {
-    const int jl = j / E;
-    const bool lower = (lane & jl) == 0;
+// Sorts N values held by one thread ascending (bitonic network; every index
+// is a compile-time constant, so the values stay in registers).
+template <int N>
+__device__ __forceinline__ void sort_asc(uint32_t (&a)[N]) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const uint64_t p = __shfl_xor_sync(kFull, x[e], jl);
-      const bool desc = ((lane * E + e) & k) == 0;
-      x[e] = (x[e] > p) == (lower == desc) ? x[e] : p;
-    }
-  }
-}
-
-// Sorts the warp's 32E keys descending (key i at lane i / E, slot i % E).
-template <int E>
-__device__ __forceinline__ void warp_sort_desc(uint64_t (&x)[E], int lane) {
+  for (int k = 2; k <= N; k <<= 1)
 #pragma unroll
-  for (int k = 2; k <= 32 * E; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1)
 #pragma unroll
-    for (int j = k >> 1; j > 0; j >>= 1) bitonic_step<E>(x, lane, k, j);
+      for (int i = 0; i < N; ++i) {
+        const int l = i ^ j;
+        if (l > i) {
+          const uint32_t x = a[i], y = a[l];
+          const bool up = (i & k) == 0;
+          a[i] = up ? min(x, y) : max(x, y);
+          a[l] = up ? max(x, y) : min(x, y);
+        }
+      }
 }
 
 template <int D, int NC, int LISTN>
@@ -375,38 +363,34 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
     tc::tmem_dealloc(tmem, Ly::TMEM_COLS);
   }
 
-  // One row at a time per warp: the kept keys (live heap slots holding a
-  // real key) become block indices, sorted ascending across the lanes and
-  // written coalesced, followed by the own block and -1 padding.
-  constexpr int E = LISTN / 32;
+  // Each thread writes its own row: the kept keys (live heap slots holding a
+  // real key) become block indices, sorted ascending in registers, followed
+  // by the own block and -1 padding.
   float best_mine = -INFINITY;
-  const int rows_here = min(32, nrows - warp * 32);
-  for (int r = 0; r < rows_here; ++r) {
-    const int rr = warp * 32 + r;
-    uint64_t y[E], top = 0ull;
+  if (row_ok) {
+    uint32_t ix[LISTN];
+    uint64_t top = 0ull;
     int kept_n = 0;
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int i = lane * E + e;
-      const uint64_t key = i < k1 ? heap[i * kSel + rr] : kKeyEmpty;
+    for (int sl = 0; sl < LISTN; ++sl) {
+      const uint64_t key = sl < k1 ? heap[sl * kSel + tid] : kKeyEmpty;
       const bool real = key != kKeyEmpty;
-      kept_n += __popc(__ballot_sync(kFull, real));
-      y[e] = real ? (key & 0xffffffffull) : 0ull;  // inverted index: larger = lower block
+      kept_n += real;
+      ix[sl] = real ? 0xffffffffu - (uint32_t)key : 0x7fffffffu;  // block index; empty slots sort last
       top = real && key > top ? key : top;
     }
+    if (top) best_mine = from_order_bits((uint32_t)(top >> 32));
+    sort_asc<LISTN>(ix);
+    int32_t* out = sel_idx + ((size_t)(t0 + tid) * h_q + h) * topk;
+    auto val = [&](int i) -> int32_t { return i < kept_n ? (int32_t)ix[i] : (i == kept_n ? my_b : -1); };
+    if ((topk & 3) == 0) {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const uint64_t o = __shfl_xor_sync(kFull, top, off);
-      top = o > top ? o : top;
-    }
-    if (lane == r && top) best_mine = from_order_bits((uint32_t)(top >> 32));
-    warp_sort_desc<E>(y, lane);
-    const int own = __shfl_sync(kFull, my_b, r);
-    int32_t* out = sel_idx + ((size_t)(t0 + rr) * h_q + h) * topk;
+      for (int i = 0; i < LISTN; i += 4)
+        if (i < topk) *reinterpret_cast<int4*>(out + i) = make_int4(val(i), val(i + 1), val(i + 2), val(i + 3));
+    } else {
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int i = lane * E + e;
-      if (i < topk) out[i] = i < kept_n ? (int32_t)(0xffffffffu - (uint32_t)y[e]) : (i == kept_n ? own : -1);
+      for (int i = 0; i < LISTN; ++i)
+        if (i < topk) out[i] = val(i);
     }
   }
 
