@@ -48,11 +48,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel source file it was taken with: a changed source voids the figure.
 # Headline workload, one timed-step launch each (profiles/dram_traffic_n64k_h16_d64_b32_k32_kconv4.md).
 NCU_TRAFFIC = {
-    "fwd_route": {"bytes": 303.11e6 + 375.30e6, "sha": "2b7aa8ef0ce7e4e7"},
-    "fwd_attn": {"bytes": 1.040e9 + 620.68e6, "sha": "f7c5118786edd477"},
-    "bwd_attn": {"bytes": 1.070e9 + 568.15e6, "sha": "7fe3d119690989cd"},
-    "conv_bwd": {"bytes": 268.50e6 + 128.18e6, "sha": "2e8a64640582a328"},
-    "fwd_centroid": {"bytes": 134.26e6 + 102.33e6, "sha": "103ae9898d36c11f"},
+    "fwd_route": {"bytes": 278.73e6 + 367.28e6, "sha": "5ebadca9177dc9a1"},
+    "fwd_attn": {"bytes": 1.2337e9 + 807.07e6, "sha": "d2ec950c614ceda1"},
+    "bwd_attn": {"bytes": 1.9366e9 + 1.0377e9, "sha": "b52f866589d7344f"},
+    "conv_bwd": {"bytes": 268.46e6 + 127.56e6, "sha": "2e8a64640582a328"},
+    "fwd_centroid": {"bytes": 134.28e6 + 102.18e6, "sha": "103ae9898d36c11f"},
 }
 
 

@@ -71,30 +71,51 @@ count_kernel(const int32_t* __restrict__ sel_idx, long long npicks, int topk, in
   }
 }
 
-// Exclusive scan of cnt[0..n) into ptr[0..n]; cursor = ptr[0..n).
+// Exclusive scan of cnt[0..n) into ptr[0..n]; cursor = ptr[0..n).  One CTA:
+// each warp owns a contiguous segment, read 32 entries at a time (coalesced);
+// pass 1 sums the segments, a scan over the warp sums gives each segment's
+// start, pass 2 re-reads the segment and writes the running prefix.
 __global__ void __launch_bounds__(kScanThreads)
 scan_kernel(const int32_t* __restrict__ cnt, int n, int32_t* __restrict__ ptr, int32_t* __restrict__ cursor) {
-  __shared__ int32_t s_sum[kScanThreads];
-  const int tid = threadIdx.x;
-  const int per = (n + kScanThreads - 1) / kScanThreads;
-  const int lo = min(tid * per, n), hi = min(lo + per, n);
-  int local = 0;
-  for (int i = lo; i < hi; ++i) local += cnt[i];
-  s_sum[tid] = local;
+  constexpr int kWarps = kScanThreads / 32;
+  __shared__ int32_t s_warp[kWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int seg = (n + kWarps - 1) / kWarps;
+  const int lo = min(warp * seg, n), hi = min(lo + seg, n);
+  int sum = 0;
+  for (int i = lo + lane; i < hi; i += 32) sum += __ldg(cnt + i);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane == 0) s_warp[warp] = sum;
   __syncthreads();
-  for (int off = 1; off < kScanThreads; off <<= 1) {
-    const int v = tid >= off ? s_sum[tid - off] : 0;
-    __syncthreads();
-    s_sum[tid] += v;
-    __syncthreads();
+  if (warp == 0) {
+    const int v = s_warp[lane];  // kWarps == 32
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    s_warp[lane] = incl - v;
+    if (lane == 31) ptr[n] = incl;
   }
-  int run = s_sum[tid] - local;
-  for (int i = lo; i < hi; ++i) {
-    ptr[i] = run;
-    cursor[i] = run;
-    run += cnt[i];
+  __syncthreads();
+  int run = s_warp[warp];
+  for (int i0 = lo; i0 < hi; i0 += 32) {
+    const int i = i0 + lane;
+    const int v = i < hi ? __ldg(cnt + i) : 0;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (i < hi) {
+      ptr[i] = run + incl - v;
+      cursor[i] = run + incl - v;
+    }
+    run += __shfl_sync(0xffffffffu, incl, 31);
   }
-  if (tid == kScanThreads - 1) ptr[n] = s_sum[tid];
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -186,18 +207,25 @@ chunk_count_kernel(const int32_t* __restrict__ sel_idx, int total_tokens, int to
 }
 
 // Per bucket: chunk counts -> exclusive prefix over chunks (in place), total
-// into cnt.
+// into cnt.  A thread reads eight chunks' counts before writing them back, so
+// its loads overlap.
 __global__ void __launch_bounds__(kThreads)
 chunk_prefix_kernel(int32_t* __restrict__ chunk_cnt, int nb_max, int nchunks, int h_kv, int32_t* __restrict__ cnt) {
+  constexpr int U = 8;
   const int b = blockIdx.x * kThreads + threadIdx.x;
   if (b >= h_kv * nb_max) return;
   const int kvh = b / nb_max, lb = b % nb_max;
   int32_t* col = chunk_cnt + (size_t)kvh * nchunks * nb_max + lb;
   int run = 0;
-  for (int c = 0; c < nchunks; ++c) {
-    const int v = col[(size_t)c * nb_max];
-    col[(size_t)c * nb_max] = run;
-    run += v;
+  for (int c0 = 0; c0 < nchunks; c0 += U) {
+    int v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) v[u] = c0 + u < nchunks ? col[(size_t)(c0 + u) * nb_max] : 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (c0 + u < nchunks) col[(size_t)(c0 + u) * nb_max] = run;
+      run += v[u];
+    }
   }
   cnt[b] = run;
 }
