@@ -253,6 +253,119 @@ chunk_fill_kernel(const int32_t* __restrict__ sel_idx, int total_tokens, int top
   }
 }
 
+// Staged fill (blocks per KV head <= kMaxStagedBuckets): the chunk's rows are
+// taken in passes of at most kStage picks.  A pass counts its picks per block
+// in shared memory, scans the counts into local bucket starts, places each
+// row id at its local slot (with its bucket as a tag) and then copies the
+// staged entries out in order: consecutive entries of one bucket go to
+// consecutive addresses, so the stores coalesce into runs instead of one
+// scattered 4-byte store per pick.  `base[b]` is where the chunk's next entry
+// for block b goes in rows[].
+constexpr int kStage = 8192;
+constexpr int kMaxStagedBuckets = 8192;
+
+__host__ __device__ constexpr size_t staged_fill_smem(int nb_max) {
+  return sizeof(int32_t) * (2 * (size_t)nb_max + 1 + kStage) + sizeof(uint16_t) * kStage;
+}
+
+// In-place exclusive scan of a[0..n) by the whole CTA (kThreads threads);
+// returns the total.  `part` holds kThreads ints of shared scratch.
+__device__ int block_exclusive_scan(int32_t* a, int n, int32_t* part) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (n + kThreads - 1) / kThreads;
+  const int lo = min(tid * per, n), hi = min(lo + per, n);
+  int sum = 0;
+  for (int i = lo; i < hi; ++i) sum += a[i];
+  int incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) part[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = lane < kThreads / 32 ? part[lane] : 0;
+    int w = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += o;
+    }
+    if (lane < kThreads / 32) part[lane] = w - v;
+    if (lane == 31) part[kThreads / 32] = w;  // total
+  }
+  __syncthreads();
+  int run = part[warp] + incl - sum;
+  for (int i = lo; i < hi; ++i) {
+    const int v = a[i];
+    a[i] = run;
+    run += v;
+  }
+  const int total = part[kThreads / 32];
+  __syncthreads();
+  return total;
+}
+
+__global__ void __launch_bounds__(kThreads)
+chunk_fill_staged_kernel(const int32_t* __restrict__ sel_idx, int total_tokens, int topk, int h_q, int group,
+                         int block_size, const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off,
+                         int batch, int nb_max, int nchunks, const int32_t* __restrict__ chunk_cnt,
+                         const int32_t* __restrict__ ptr, int32_t* __restrict__ rows) {
+  extern __shared__ __align__(16) int32_t sm_fill[];
+  int32_t* base = sm_fill;                  // [nb_max]
+  int32_t* lc = base + nb_max;              // [nb_max + 1]: counts -> local starts -> cursors
+  int32_t* stage = lc + nb_max + 1;         // [kStage]
+  uint16_t* tag = reinterpret_cast<uint16_t*>(stage + kStage);  // [kStage]
+  __shared__ int32_t part[kThreads / 32 + 1];
+  const int c = blockIdx.x, kvh = blockIdx.y;
+  const int tid = threadIdx.x;
+  const int32_t* src = chunk_cnt + ((size_t)kvh * nchunks + c) * nb_max;
+  const int32_t* bptr = ptr + (size_t)kvh * nb_max;
+  for (int b = tid; b < nb_max; b += kThreads) base[b] = __ldg(bptr + b) + __ldg(src + b);
+  const int ta = c * kChunkTokens;
+  const int ntok = max(0, min(kChunkTokens, total_tokens - ta));
+  const int seq_end = __ldg(cu + batch);
+  const int nrows = ntok * group;
+  const int pass_rows = max(1, kStage / topk);
+  for (int r0 = 0; r0 < nrows; r0 += pass_rows) {
+    const int r1 = min(nrows, r0 + pass_rows);
+    for (int b = tid; b <= nb_max; b += kThreads) lc[b] = 0;
+    __syncthreads();
+    // 1. count this pass's picks per block (invalid entries were reported by
+    //    the count pass and are skipped here)
+    for (int r = r0 + tid; r < r1; r += kThreads) {
+      int row, bb, own;
+      if (!chunk_row(r, ntok, ta, kvh, group, h_q, block_size, cu, blk_off, batch, seq_end, row, bb, own)) continue;
+      for_row_picks<false>(sel_idx, row, topk, own, nullptr, [&](int, int j) { atomicAdd(lc + bb + j, 1); });
+    }
+    __syncthreads();
+    // 2. local bucket starts
+    const int total = block_exclusive_scan(lc, nb_max, part);
+    // 3. stage each row id at its local slot
+    for (int r = r0 + tid; r < r1; r += kThreads) {
+      int row, bb, own;
+      if (!chunk_row(r, ntok, ta, kvh, group, h_q, block_size, cu, blk_off, batch, seq_end, row, bb, own)) continue;
+      for_row_picks<false>(sel_idx, row, topk, own, nullptr, [&](int, int j) {
+        const int slot = atomicAdd(lc + bb + j, 1);
+        stage[slot] = row;
+        tag[slot] = (uint16_t)(bb + j);
+      });
+    }
+    __syncthreads();
+    // 4. copy out in order; lc[b] is now the end of bucket b's local run, so
+    //    the run starts at lc[b - 1]
+    for (int i = tid; i < total; i += kThreads) {
+      const int b = tag[i];
+      const int start = b > 0 ? lc[b - 1] : 0;
+      rows[base[b] + (i - start)] = stage[i];
+    }
+    __syncthreads();
+    for (int b = tid; b < nb_max; b += kThreads) base[b] += lc[b] - (b > 0 ? lc[b - 1] : 0);
+    __syncthreads();
+  }
+}
+
 }  // namespace
 
 size_t index_chunk_ints(int total_tokens, int h_kv, int nb_max) {
@@ -286,6 +399,16 @@ cudaError_t launch_build_index(const int32_t* sel_idx, const SeqPlan& p, int h_q
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     scan_kernel<<<1, kScanThreads, 0, st>>>(cnt, nbk, ptr, cursor);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (p.nb_max <= kMaxStagedBuckets && topk <= kStage) {
+      const size_t smem2 = staged_fill_smem(p.nb_max);
+      if ((e = cudaFuncSetAttribute(chunk_fill_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem2)) != cudaSuccess)
+        return e;
+      chunk_fill_staged_kernel<<<grid, kThreads, smem2, st>>>(sel_idx, p.total_tokens, topk, h_q, group, block_size,
+                                                              p.cu, p.blk_off, p.batch, p.nb_max, nchunks, chunk_cnt,
+                                                              ptr, rows);
+      return cudaGetLastError();
+    }
     chunk_fill_kernel<<<grid, kThreads, smem, st>>>(sel_idx, p.total_tokens, topk, h_q, group, block_size, p.cu,
                                                     p.blk_off, p.batch, p.nb_max, nchunks, chunk_cnt, ptr, rows,
                                                     status);
