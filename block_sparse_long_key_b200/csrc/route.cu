@@ -231,8 +231,36 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
     int pos = 0;
     bool done = false;
     uint64_t root = key;  // the new minimum: the key itself or the smaller child of the root
+    // Two levels per step: the children and all four grandchildren are
+    // loaded together (none depends on the first decision), which halves the
+    // chain of dependent shared-memory loads.
+    int lvl = 0;
 #pragma unroll
-    for (int lvl = 0; lvl < kHeapDepth; ++lvl) {
+    for (; lvl + 1 < kHeapDepth; lvl += 2) {
+      const int c1 = 2 * pos + 1, g1 = 2 * c1 + 1;
+      const uint64_t a0 = heap[c1 * kSel + tid], a1 = heap[(c1 + 1) * kSel + tid];
+      const uint64_t b0 = heap[g1 * kSel + tid], b1 = heap[(g1 + 1) * kSel + tid];
+      const uint64_t b2 = heap[(g1 + 2) * kSel + tid], b3 = heap[(g1 + 3) * kSel + tid];
+      const bool left = a0 < a1;
+      const uint64_t km = left ? a0 : a1;
+      if (!done && km < key) {
+        heap[pos * kSel + tid] = km;
+        if (lvl == 0) root = km;
+        pos = left ? c1 : c1 + 1;
+      } else {
+        done = true;
+      }
+      const uint64_t d0 = left ? b0 : b2, d1 = left ? b1 : b3;  // children of the chosen child
+      const bool left2 = d0 < d1;
+      const uint64_t km2 = left2 ? d0 : d1;
+      if (!done && km2 < key) {
+        heap[pos * kSel + tid] = km2;
+        pos = 2 * pos + (left2 ? 1 : 2);
+      } else {
+        done = true;
+      }
+    }
+    if (lvl < kHeapDepth) {
       const int c1 = 2 * pos + 1;
       const uint64_t k1v = heap[c1 * kSel + tid];
       const uint64_t k2v = heap[(c1 + 1) * kSel + tid];
@@ -242,8 +270,6 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
         heap[pos * kSel + tid] = km;
         if (lvl == 0) root = km;
         pos = left ? c1 : c1 + 1;
-      } else {
-        done = true;
       }
     }
     heap[pos * kSel + tid] = key;
