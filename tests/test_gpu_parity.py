@@ -118,6 +118,44 @@ def test_block_index_matches_oracle(dev, case):
     assert ptr[-1] == sum(len(v) for v in want.values())
 
 
+def _random_picks(seqlen, hq, B, seed):
+    """Valid picks for every row of one sequence: two distinct past blocks
+    (fewer when there are fewer), then the own block, then -1."""
+    rng = np.random.default_rng(seed)
+    own = np.repeat(np.arange(seqlen) // B, hq)
+    sel = np.full((seqlen * hq, 3), -1, dtype=np.int32)
+    a = rng.integers(0, np.maximum(own, 1))
+    b = (a + 1 + rng.integers(0, np.maximum(own - 1, 1))) % np.maximum(own, 1)
+    two = own >= 2
+    sel[two, 0] = np.minimum(a, b)[two]
+    sel[two, 1] = np.maximum(a, b)[two]
+    sel[two, 2] = own[two]
+    one = own == 1
+    sel[one, 0], sel[one, 1] = 0, 1
+    sel[own == 0, 0] = 0
+    return sel.reshape(seqlen, hq, 3)
+
+
+# Blocks per KV head: staged fill (<= 8192), shared-memory cursors (<= 16384),
+# one global atomic per pick (> 16384).
+@pytest.mark.parametrize("seqlen", [100_000, 200_000, 300_000])
+def test_block_index_large_block_counts(dev, seqlen):
+    B, hq, hkv = 16, 2, 1
+    sel = _random_picks(seqlen, hq, B, seed=seqlen)
+    cu = np.array([0, seqlen], dtype=np.int32)
+    ptr, rows = moba.build_index(torch.from_numpy(sel).to(dev), torch.from_numpy(cu).to(dev), hkv, B)
+    torch.cuda.synchronize()
+    want = orc.block_index(sel, cu, B, hkv)
+    ptr, rows = ptr.cpu().numpy(), rows.cpu().numpy()
+    nb = seqlen // B + 1
+    assert ptr[-1] == sum(len(v) for v in want.values())
+    for (kvh, gb), lst in want.items():
+        b = kvh * nb + gb
+        assert sorted(rows[ptr[b]:ptr[b + 1]].tolist()) == lst, (kvh, gb)
+    assert all(ptr[kvh * nb + gb + 1] == ptr[kvh * nb + gb] for kvh in range(hkv) for gb in range(nb)
+               if (kvh, gb) not in want)
+
+
 @pytest.mark.parametrize("case", SMALL, ids=_ids)
 def test_backward_matches_oracle(dev, case):
     w, x = _inputs(case)
