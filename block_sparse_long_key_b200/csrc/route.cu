@@ -22,15 +22,17 @@
 // of the fp32 centroid, while the four selecting warps work on earlier chunks
 // (mbarrier hand-offs per score tile, no block-wide barrier per chunk).
 // Thread t owns query row t, which is TMEM lane t: tcgen05.ld hands it that
-// row's NC scores in registers.  Scores above the
-// thread's running threshold (the worst of its current k-1 best) go to a
-// small per-thread candidate buffer in shared memory; the whole warp flushes
-// the buffers together.  The k-1 kept entries form a binary min-heap of
-// 64-bit keys (order-preserving score bits << 32 | ~block index, so a larger
-// key is a better block: higher score, then lower index) in shared memory
-// ([slot][thread], bank-conflict free); admitting a candidate replaces the
-// root and sifts it down a fixed log2(k) levels whatever the data (a sorted
-// list would shift up to k-1 entries, and a warp pays for its slowest lane).
+// row's NC scores in registers.  Scores above the thread's running threshold
+// (the worst of its current k-1 best) go to a small per-thread candidate
+// buffer in shared memory; the whole warp flushes the buffers together.  The
+// k-1 kept entries form a binary min-heap of 64-bit keys (order-preserving
+// score bits << 32 | ~block index, so a larger key is a better block: higher
+// score, then lower index) in shared memory ([slot][thread], bank-conflict
+// free); admitting a candidate replaces the root and sifts it down a fixed
+// log2(k) levels whatever the data, two levels per step (a sorted list would
+// shift up to k-1 entries, and a warp pays for its slowest lane).  At the
+// end each thread sorts its row's kept block indices in registers and writes
+// the row.
 //
 // Side outputs for the forward: mref = a lower bound of the query's largest
 // attention logit, max(best kept score, q_i.k_i) / sqrt(d) (a block mean never
