@@ -229,9 +229,11 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   }
 
   // Admit a key above the root: replace the root and sift it down.
-  auto admit = [&](uint64_t key) {
+  // Admits `key` when `go` (branch-free: a thread with nothing to admit
+  // walks the same instructions with every store switched off).
+  auto admit = [&](uint64_t key, bool go) {
     int pos = 0;
-    bool done = false;
+    bool done = !go;
     uint64_t root = key;  // the new minimum: the key itself or the smaller child of the root
     // Two levels per step: the children and all four grandchildren are
     // loaded together (none depends on the first decision), which halves the
@@ -274,20 +276,21 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
         pos = left ? c1 : c1 + 1;
       }
     }
-    heap[pos * kSel + tid] = key;
-    root_key = root;
-    tau = from_order_bits((uint32_t)(root >> 32));
+    if (go) {
+      heap[pos * kSel + tid] = key;
+      root_key = root;
+      tau = from_order_bits((uint32_t)(root >> 32));
+    }
   };
   // One round: every thread with buffered keys admits its latest one (full
   // keys are compared, so the order of admission does not matter).  Rounds
   // run only while some thread's buffer is close to full, so most threads
   // have work in each of them.
   auto flush_round = [&]() {
-    if (cnt > 0) {
-      --cnt;
-      const uint64_t key = bk[cnt * kSel + tid];
-      if (key > root_key) admit(key);
-    }
+    const bool has = cnt > 0;
+    cnt -= has ? 1 : 0;
+    const uint64_t key = bk[cnt * kSel + tid];  // slot 0 when empty: read, not used
+    admit(key, has && key > root_key);
   };
 
   // Selection on one chunk's scores: those above the row's threshold go to
