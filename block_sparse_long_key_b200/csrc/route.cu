@@ -307,7 +307,10 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
         const int j = jbase + col;
         // Blocks arrive in ascending j, so a score equal to tau (the root's,
         // which has a lower index) never wins: the strict test is exact.
-        if (j < my_b && x > tau) bk[(cnt++) * kSel + tid] = make_key(x, j);
+        // Branch-free: slot cnt is free (cnt < kBuf here), so the key is
+        // stored either way and only counted when it passes.
+        bk[cnt * kSel + tid] = make_key(x, j);
+        cnt += (j < my_b && x > tau) ? 1 : 0;
       }
     }
   };
