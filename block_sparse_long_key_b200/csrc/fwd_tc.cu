@@ -75,7 +75,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
   using Ly = FwdTcLayout<D, BLK>;
   constexpr int OS = oacc_stride(D);
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, derived from the shared array by pointer
+  // arithmetic so that accesses through it stay shared-memory accesses.
+  unsigned char* sm = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
   const uint32_t sbase = smem_u32(sm);
   const uint32_t mb_s = sbase + Ly::MB_OFF, mb_o = mb_s + 8, mb_q = mb_s + 16;
 

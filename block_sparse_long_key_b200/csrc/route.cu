@@ -124,7 +124,9 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   // deepest internal node still lie below LISTN - 1).
   constexpr int kHeapDepth = LISTN == 64 ? 5 : (LISTN == 32 ? 4 : (LISTN == 16 ? 3 : 2));
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, derived from the shared array by pointer
+  // arithmetic so that accesses through it stay shared-memory accesses.
+  unsigned char* sm = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
   const uint32_t sbase = smem_u32(sm);
   uint64_t* heap = reinterpret_cast<uint64_t*>(sm + Ly::HP_OFF);
   uint64_t* bk = reinterpret_cast<uint64_t*>(sm + Ly::BK_OFF);
