@@ -18,9 +18,12 @@
 //      The next tile's gather starts here: the Q tile is free once S is.
 //   4. One thread issues O = P V_j (M = 128, N = d, K = B; V_j read
 //      N-major) into the columns S used.
-//   5. Each thread reads its O row and adds it, and l, to the query's fp32
-//      accumulator row (O, d floats; l in its own array) with 16-byte
-//      vector reductions (lane pairs cover whole 32-byte sectors).
+//   5. Each thread adds its row's l to the query's fp32 l; the O rows leave
+//      through the (now free) P tile: each warp stages column pieces of its
+//      32 rows there, then 4 (8 at B = 64) lanes cover one 64- (128-) byte
+//      row piece per 16-byte vector reduction into the query's fp32
+//      accumulator row (d floats), so an instruction touches 8 (4) rows
+//      instead of 16.
 // The merge of a query's k blocks is therefore a plain sum; finalize divides
 // by l.  A CTA needs ~33 KB of shared memory and 64 TMEM columns at d = 64,
 // so several share an SM and overlap their phases.  Every mbarrier wait is
@@ -236,34 +239,39 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
       atomicAdd(lacc + rid, l);
       if (mx - mr_c > kOverflowLog2) flag[rid] = 1;
     }
-    const int prow = __shfl_xor_sync(0xffffffffu, rid, 1);  // the lane pair's other row
-    const bool even = (lane & 1) == 0;
-    const int r1 = even ? rid : prow, r2 = even ? prow : rid;  // even lane's row, odd lane's row
+    // O rows leave through the (now free) P tile: each warp stages CPP-column
+    // pieces of its 32 rows, then LPR lanes cover one row piece per 16-byte
+    // reduction (fewer rows per instruction than one lane per row).
+    {
+      constexpr int CPP = (int)(Ly::P_BYTES / 4) / (32 * 4);  // columns per pass
+      constexpr int RB = CPP * 4;                              // bytes per staged row piece
+      constexpr int LPR = RB / 16;                             // lanes per row piece
+      constexpr int RPI = 32 / LPR;                            // rows per instruction
+      static_assert(32 % CPP == 0 && LPR >= 4, "staging geometry");
+      unsigned char* stg = sm + Ly::P_OFF + warp * (32 * RB);
+      auto swz = [](int row, int c) { return LPR == 8 ? (c ^ (row & 7)) : (c ^ ((row >> 1) & 3)); };
 #pragma unroll
-    for (int h = 0; h < D / 32; ++h) {
-      uint32_t ov[32];
-      tc::tmem_ld32(tmem + lane_base + h * 32, ov);
-      tc::tmem_ld_wait();
+      for (int h = 0; h < D / 32; ++h) {
+        uint32_t ov[32];
+        tc::tmem_ld32(tmem + lane_base + h * 32, ov);
+        tc::tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        // Even lane: columns 8j..8j+3 of both rows; odd lane: 8j+4..8j+7.
-        float send[4], mine[4], got[4], v1[4], v2[4];
+        for (int ps = 0; ps < 32 / CPP; ++ps) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float lo = __uint_as_float(ov[8 * j + u]), hi = __uint_as_float(ov[8 * j + 4 + u]);
-          send[u] = even ? hi : lo;
-          mine[u] = even ? lo : hi;
+          for (int c = 0; c < LPR; ++c)
+            *reinterpret_cast<float4*>(stg + lane * RB + (swz(lane, c) << 4)) =
+                make_float4(__uint_as_float(ov[ps * CPP + 4 * c]), __uint_as_float(ov[ps * CPP + 4 * c + 1]),
+                            __uint_as_float(ov[ps * CPP + 4 * c + 2]), __uint_as_float(ov[ps * CPP + 4 * c + 3]));
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 32 / RPI; ++i) {
+            const int rl = i * RPI + lane / LPR, c = lane % LPR;
+            const float4 val = *reinterpret_cast<const float4*>(stg + rl * RB + (swz(rl, c) << 4));
+            const int row = __shfl_sync(0xffffffffu, rid, rl);
+            if (row >= 0) red_add_v4(oacc + (size_t)row * OS + h * 32 + ps * CPP + c * 4, val.x, val.y, val.z, val.w);
+          }
+          __syncwarp();
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) got[u] = __shfl_xor_sync(0xffffffffu, send[u], 1);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          v1[u] = even ? mine[u] : got[u];
-          v2[u] = even ? got[u] : mine[u];
-        }
-        const int col = h * 32 + 8 * j + (even ? 0 : 4);
-        if (r1 >= 0) red_add_v4(oacc + (size_t)r1 * OS + col, v1[0], v1[1], v1[2], v1[3]);
-        if (r2 >= 0) red_add_v4(oacc + (size_t)r2 * OS + col, v2[0], v2[1], v2[2], v2[3]);
       }
     }
     tc::fence_before_sync();
