@@ -19,14 +19,13 @@
 //   4. One thread issues O = P V_j (M = 128, N = d, K = B; V_j read
 //      N-major) into the columns S used.
 //   5. Each thread adds its row's l to the query's fp32 l; the O rows leave
-//      through the (now free) P tile: each warp stages column pieces of its
-//      32 rows there, then 4 (8 at B = 64) lanes cover one 64- (128-) byte
-//      row piece per 16-byte vector reduction into the query's fp32
-//      accumulator row (d floats), so an instruction touches 8 (4) rows
-//      instead of 16.
+//      through the (now free) P tile: each warp stages 32-column pieces of
+//      its 32 rows there, then 8 lanes cover one 128-byte row piece per
+//      16-byte vector reduction into the query's fp32 accumulator row (d
+//      floats), so an instruction touches 4 rows, not 16 (one line each).
 // The merge of a query's k blocks is therefore a plain sum; finalize divides
-// by l.  A CTA needs ~33 KB of shared memory and 64 TMEM columns at d = 64,
-// so several share an SM and overlap their phases.  Every mbarrier wait is
+// by l.  A CTA needs ~41 KB of shared memory and 64 TMEM columns at d = 64,
+// so five share an SM and overlap their phases.  Every mbarrier wait is
 // bounded; a timeout sets MOBA_STATUS_TIMEOUT and the CTA winds down.
 #include "common.cuh"
 #include "launch.h"
@@ -52,7 +51,10 @@ struct FwdTcLayout {
   static constexpr uint32_t V_OFF = K_OFF + KB * KV_REGION;
   static constexpr uint32_t Q_OFF = V_OFF + KB * KV_REGION;
   static constexpr uint32_t P_OFF = Q_OFF + KB * Q_REGION;
-  static constexpr uint32_t MB_OFF = P_OFF + P_BYTES;    // mbS, mbO, mbQ
+  // The P tile, grown to 16 KB where it is smaller, doubles as the staging
+  // area of the O reductions (32 rows x 128 bytes per warp).
+  static constexpr uint32_t STG_BYTES = P_BYTES < 16384 ? 16384 : P_BYTES;
+  static constexpr uint32_t MB_OFF = P_OFF + STG_BYTES;    // mbS, mbO, mbQ
   static constexpr uint32_t HOLD_OFF = MB_OFF + 24;
   static constexpr uint32_t BYTES = HOLD_OFF + 16;
   // Tensor memory: S (B columns), later overwritten by O (D columns).
@@ -243,7 +245,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
     // pieces of its 32 rows, then LPR lanes cover one row piece per 16-byte
     // reduction (fewer rows per instruction than one lane per row).
     {
-      constexpr int CPP = (int)(Ly::P_BYTES / 4) / (32 * 4);  // columns per pass
+      constexpr int CPP = (int)(Ly::STG_BYTES / 4) / (32 * 4);  // columns per pass
       constexpr int RB = CPP * 4;                              // bytes per staged row piece
       constexpr int LPR = RB / 16;                             // lanes per row piece
       constexpr int RPI = 32 / LPR;                            // rows per instruction
