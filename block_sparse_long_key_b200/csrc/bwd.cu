@@ -300,8 +300,8 @@ bwd_attn_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
 // D_i = sum_c dO_ic O_ic (fp32) and dQ accumulator zeroing; D/8 lanes per row.
 template <int D>
 __global__ void __launch_bounds__(256)
-bwd_pre_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout, long long nrows,
-               float* __restrict__ dsum, float* __restrict__ dqacc) {
+bwd_pre_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout, const float* __restrict__ lse,
+               long long nrows, float* __restrict__ dsum, float2* __restrict__ stat, float* __restrict__ dqacc) {
   constexpr int LPR = D / 8;
   const long long nthreads = (long long)gridDim.x * 256;
   const long long total = nrows * LPR;
@@ -321,7 +321,10 @@ bwd_pre_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout, long
 #pragma unroll
     for (int off = LPR / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (ok) {
-      if (i % LPR == 0) dsum[i / LPR] = acc;
+      if (i % LPR == 0) {
+        dsum[i / LPR] = acc;
+        stat[i / LPR] = make_float2(__ldg(lse + i / LPR), acc);  // one 8-byte load per row downstream
+      }
       float4* z = reinterpret_cast<float4*>(dqacc) + 2 * i;
       z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
       z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -357,15 +360,15 @@ cudaError_t launch_bwd_t(const bf16* q, const bf16* k, const bf16* v, const bf16
 
 }  // namespace
 
-cudaError_t launch_bwd_pre(const bf16* out, const bf16* dout, int nrows, int d, float* dsum, float* dqacc,
-                           cudaStream_t st) {
+cudaError_t launch_bwd_pre(const bf16* out, const bf16* dout, const float* lse, int nrows, int d, float* dsum,
+                           float2* stat, float* dqacc, cudaStream_t st) {
   const long long n = (long long)nrows * (d / 8);
   if (n == 0) return cudaSuccess;
   const int grid = (int)std::min<long long>((n + 255) / 256, 148LL * 32);
   if (d == 64)
-    bwd_pre_kernel<64><<<grid, 256, 0, st>>>(out, dout, nrows, dsum, dqacc);
+    bwd_pre_kernel<64><<<grid, 256, 0, st>>>(out, dout, lse, nrows, dsum, stat, dqacc);
   else
-    bwd_pre_kernel<128><<<grid, 256, 0, st>>>(out, dout, nrows, dsum, dqacc);
+    bwd_pre_kernel<128><<<grid, 256, 0, st>>>(out, dout, lse, nrows, dsum, stat, dqacc);
   return cudaGetLastError();
 }
 

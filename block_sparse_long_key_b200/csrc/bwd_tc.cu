@@ -80,7 +80,7 @@ __device__ __forceinline__ uint32_t p_offset(int r, int c) {
 template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads)
 bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__ k, const bf16* __restrict__ v,
-              const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ lse, const float* __restrict__ dsum,
+              const __grid_constant__ CUtensorMap tm_do, const float2* __restrict__ stat,
               const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch, int nb_max,
               int h_q, int h_kv, int lead, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
               float* __restrict__ dqacc, bf16* __restrict__ dk, bf16* __restrict__ dv,
@@ -158,7 +158,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
   if (warp == 0) tc::tmem_alloc(sbase + Ly::HOLD_OFF, Ly::TMEM_COLS);
   cp_async_commit();
   int rid = meta_rid(0), nrid = -1;
-  float lse_c = rid >= 0 ? __ldg(lse + rid) : 0.f, dsum_c = rid >= 0 ? __ldg(dsum + rid) : 0.f;
+  const float2 st0 = rid >= 0 ? __ldg(stat + rid) : make_float2(0.f, 0.f);  // (LSE, D) of the row
+  float lse_c = st0.x, dsum_c = st0.y;
   float lse_n = 0.f, dsum_n = 0.f;
   tc::fence_before_sync();
   __syncthreads();
@@ -239,8 +240,11 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
         }
       }
     }
-    lse_n = nrid >= 0 ? __ldg(lse + nrid) : 0.f;
-    dsum_n = nrid >= 0 ? __ldg(dsum + nrid) : 0.f;
+    {
+      const float2 st1 = nrid >= 0 ? __ldg(stat + nrid) : make_float2(0.f, 0.f);
+      lse_n = st1.x;
+      dsum_n = st1.y;
+    }
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
@@ -357,7 +361,7 @@ bool bwd_tc_supported(int d, int block_size) {
 }
 
 cudaError_t launch_bwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const CUtensorMap& tm_do,
-                          const float* lse, const float* dsum, const SeqPlan& p, const int32_t* ptr,
+                          const float2* stat, const SeqPlan& p, const int32_t* ptr,
                           const int32_t* rows, int h_q, int h_kv, int d, int block_size, float* dqacc, bf16* dk,
                           bf16* dv, int32_t* status, cudaStream_t st) {
 #define MOBA_BWD_TC(DD, BB)                                                                                  \
@@ -368,7 +372,7 @@ cudaError_t launch_bwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v,
     if (e != cudaSuccess) return e;                                                                          \
     if (p.nb_max == 0) return cudaSuccess;                                                                   \
     const int lead = bucket_lead((long long)p.total_tokens * (h_q / h_kv), DD * 4);                          \
-    kern<<<dim3(p.nb_max * h_kv), kThreads, smem, st>>>(tm_q, k, v, tm_do, lse, dsum, p.cu, p.blk_off, p.batch, \
+    kern<<<dim3(p.nb_max * h_kv), kThreads, smem, st>>>(tm_q, k, v, tm_do, stat, p.cu, p.blk_off, p.batch, \
                                                        p.nb_max, h_q, h_kv, lead, ptr, rows, dqacc, dk, dv,   \
                                                        status);                                                \
     return cudaGetLastError();                                                                               \

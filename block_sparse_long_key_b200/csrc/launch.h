@@ -88,8 +88,10 @@ cudaError_t launch_fwd_fallback(const bf16* q, const bf16* k, const bf16* v, con
                                 int d, int block_size, int topk, bf16* out, float* lse,
                                 cudaStream_t st);
 
-cudaError_t launch_bwd_pre(const bf16* out, const bf16* dout, int nrows, int d, float* dsum,
-                           float* dqacc, cudaStream_t st);
+// dsum[row] = D_i = dO_i . O_i; stat[row] = (LSE_i, D_i) for the tcgen05
+// backward (one 8-byte load per gathered row); zeroes the dQ accumulator.
+cudaError_t launch_bwd_pre(const bf16* out, const bf16* dout, const float* lse, int nrows, int d, float* dsum,
+                           float2* stat, float* dqacc, cudaStream_t st);
 
 cudaError_t launch_bwd_attn(const bf16* q, const bf16* k, const bf16* v, const bf16* dout,
                             const float* lse, const float* dsum, const SeqPlan& p, const int32_t* ptr,
@@ -101,7 +103,7 @@ cudaError_t launch_bwd_attn(const bf16* q, const bf16* k, const bf16* v, const b
 // make_row_map over q and dout as T*H_q rows.
 bool bwd_tc_supported(int d, int block_size);
 cudaError_t launch_bwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const CUtensorMap& tm_do,
-                          const float* lse, const float* dsum, const SeqPlan& p, const int32_t* ptr,
+                          const float2* stat, const SeqPlan& p, const int32_t* ptr,
                           const int32_t* rows, int h_q, int h_kv, int d, int block_size, float* dqacc, bf16* dk,
                           bf16* dv, int32_t* status, cudaStream_t st);
 

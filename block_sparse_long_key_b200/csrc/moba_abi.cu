@@ -108,6 +108,7 @@ struct BwdBufs {
   int32_t* rows;
   int32_t* chunk_cnt;
   float* dsum;
+  float2* stat;  // (LSE, D) per row for the tcgen05 backward
   float* dqacc;
   float* dw_part;  // per-block key-conv dW partials (width <= 8)
 };
@@ -124,6 +125,7 @@ BwdBufs carve_bwd(Carve& c, const moba_shape* s) {
   const size_t nch = moba::index_chunk_ints(s->total_tokens, s->h_kv, nb_max_of(s));
   b.chunk_cnt = nch ? c.take<int32_t>(nch) : nullptr;
   b.dsum = c.take<float>(nrow);
+  b.stat = c.take<float2>(nrow);
   b.dqacc = c.take<float>(nrow * s->head_dim);
   b.dw_part = c.take<float>((size_t)s->h_kv * nb_max_of(s) * s->head_dim * 8);
   return b;
@@ -326,15 +328,15 @@ int moba_backward(const void* q, const void* k, const void* v, const void* out, 
   }
   STAGE_END(MOBA_STAGE_BWD_INDEX);
   STAGE_BEGIN(MOBA_STAGE_BWD_PRE);
-  MOBA_TRY(moba::launch_bwd_pre(static_cast<const bf16*>(out), static_cast<const bf16*>(dout), T * hq, d, b.dsum,
-                                b.dqacc, st));
+  MOBA_TRY(moba::launch_bwd_pre(static_cast<const bf16*>(out), static_cast<const bf16*>(dout), lse, T * hq, d,
+                                b.dsum, b.stat, b.dqacc, st));
   STAGE_END(MOBA_STAGE_BWD_PRE);
   STAGE_BEGIN(MOBA_STAGE_BWD_ATTN);
   CUtensorMap tm_q, tm_do;
   if (moba::bwd_tc_supported(d, shape->block_size) &&
       moba::make_row_map(&tm_q, q, (unsigned long long)T * hq, d) == cudaSuccess &&
       moba::make_row_map(&tm_do, dout, (unsigned long long)T * hq, d) == cudaSuccess) {
-    MOBA_TRY(moba::launch_bwd_tc(tm_q, static_cast<const bf16*>(k), static_cast<const bf16*>(v), tm_do, lse, b.dsum,
+    MOBA_TRY(moba::launch_bwd_tc(tm_q, static_cast<const bf16*>(k), static_cast<const bf16*>(v), tm_do, b.stat,
                                  plan, ptr, rows, hq, hkv, d, shape->block_size, b.dqacc, static_cast<bf16*>(dk),
                                  static_cast<bf16*>(dv), b.plan.status, st));
   } else {
