@@ -48,11 +48,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel source file it was taken with: a changed source voids the figure.
 # Headline workload, one timed-step launch each (profiles/dram_traffic_n64k_h16_d64_b32_k32_kconv4.md).
 NCU_TRAFFIC = {
-    "fwd_route": {"bytes": 277.81e6 + 366.40e6, "sha": "41a06d3978d3dcd1"},
-    "fwd_attn": {"bytes": 1.2353e9 + 803.85e6, "sha": "2e5f5c6270a8f460"},
-    "bwd_attn": {"bytes": 1.9661e9 + 1.0500e9, "sha": "dc3fde97bc979a55"},
-    "conv_bwd": {"bytes": 268.51e6 + 127.47e6, "sha": "2e8a64640582a328"},
-    "fwd_centroid": {"bytes": 134.25e6 + 104.00e6, "sha": "103ae9898d36c11f"},
+    "fwd_route": {"bytes": 278.41e6 + 366.40e6, "sha": "41a06d3978d3dcd1"},
+    "fwd_attn": {"bytes": 1.1735e9 + 720.60e6, "sha": "87cebeb37e249bda"},
+    "bwd_attn": {"bytes": 1.9499e9 + 1.0257e9, "sha": "fd77383753980c5b"},
+    "conv_bwd": {"bytes": 268.46e6 + 126.76e6, "sha": "2e8a64640582a328"},
+    "fwd_centroid": {"bytes": 134.25e6 + 102.10e6, "sha": "103ae9898d36c11f"},
 }
 
 
