@@ -15,7 +15,7 @@ as summarised on the lowest.today pages (Italian: "Ottimizzazione della
 Mixture of Block Attention"; German: "Optimierung von Mixture of Block
 Attention").  Section names below are the Italian page's.
 
-Readings of points the pages leave open (each is listed again in the design doc):
+Readings of points the pages leave open:
 
 * Candidate blocks: a query scores only the strictly earlier blocks of its
   own sequence; its own block is always kept and counts toward ``topk``.
