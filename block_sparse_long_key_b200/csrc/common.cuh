@@ -42,7 +42,7 @@ __device__ __forceinline__ int upper_seq(const int32_t* off, int n, int x) {
 struct BucketOrder {
   int gb, kvh;
 };
-__device__ __forceinline__ BucketOrder bucket_order(int L, int nb_max, int h_kv, int lead) {
+__host__ __device__ __forceinline__ BucketOrder bucket_order(int L, int nb_max, int h_kv, int lead) {
   lead = lead < h_kv ? lead : h_kv;
   const int big = nb_max / 8 > 1 ? nb_max / 8 : 1;
   const int small = nb_max - big;
