@@ -28,7 +28,9 @@
  *  Every pointer is a device pointer owned by the caller, 16-byte aligned
  *  (the workspace: 256-byte aligned).  The library allocates no memory, keeps
  *  no state between calls (apart from the optional per-thread stage-timing
- *  table of moba_set_stage_events) and never synchronises: each call only enqueues
+ *  table of moba_set_stage_events, a cached driver entry point used to build
+ *  TMA tensor maps on the host, and the static device scratch of
+ *  moba_build_index_noalloc) and never synchronises: each call only enqueues
  *  kernels on `stream` (a cudaStream_t; NULL = legacy default stream) and
  *  returns.  Argument errors are reported synchronously by the return code;
  *  data-dependent errors found on the device (bad cu_seqlens, out-of-range
