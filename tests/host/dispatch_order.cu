@@ -1,12 +1,13 @@
 // Host check of the attention kernels' CTA dispatch order (bucket_order):
 // for every shape and lead, the grid visits each (key block, KV head) once,
 // head h's first nb_max / 8 blocks come `lead` head-windows before its other
-// blocks, and lead = 0 is plain head-major order.  Prints "ok" or the first
-// failure.
+// blocks, and lead = 0 is plain head-major order; bucket_lead's choices on
+// a few head sizes.  Prints "ok" or the first failure.
 #include <cstdio>
 #include <vector>
 
 #include "common.cuh"
+#include "launch.h"
 
 int main() {
   const int nbs[] = {1, 2, 3, 7, 8, 9, 16, 100, 2049, 4097};
@@ -46,6 +47,23 @@ int main() {
           }
         }
       }
+  // The lead: as many head windows as let the extra heads' accumulators
+  // share half of L2 with the current head's, at most 2.
+  struct LeadCase { long long rows; int row_bytes, want; };
+  const LeadCase lc[] = {
+      {65536, 64 * 4 + 4, 2},        // 17 MB per head (N = 64K, d = 64)
+      {16384, 128 * 4 + 4, 2},       // 8.5 MB (N = 16K, d = 128)
+      {262144, 128 * 4 + 4, 0},      // 135 MB (N = 256K, d = 128)
+      {122880 * 4, 128 * 4 + 4, 0},  // GQA 4:1, 254 MB per KV head
+      {40000, 256 * 4, 0},           // 41 MB: one extra head would not fit
+      {30000, 256 * 4, 1},           // 31 MB
+      {0, 256, 0}};
+  for (const LeadCase& c : lc)
+    if (moba::bucket_lead(c.rows, c.row_bytes) != c.want) {
+      std::printf("bucket_lead(%lld, %d) = %d, want %d\n", c.rows, c.row_bytes, moba::bucket_lead(c.rows, c.row_bytes),
+                  c.want);
+      return 1;
+    }
   std::printf("ok\n");
   return 0;
 }

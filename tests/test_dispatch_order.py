@@ -13,7 +13,7 @@ CSRC = os.path.join(HERE, "..", "block_sparse_long_key_b200", "csrc")
 
 
 @pytest.mark.skipif(shutil.which("nvcc") is None, reason="needs nvcc")
-def test_bucket_order_visits_every_bucket_once_long_blocks_first():
+def test_bucket_order_and_lead():
     with tempfile.TemporaryDirectory() as td:
         exe = os.path.join(td, "dispatch_order")
         subprocess.run(["nvcc", "-std=c++17", "-O1", "-I" + CSRC, os.path.join(HERE, "host", "dispatch_order.cu"),
