@@ -305,7 +305,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
 }  // namespace
 
 bool fwd_tc_supported(int d, int block_size) {
-  return (d == 64 && block_size == 32) || (d == 128 && (block_size == 32 || block_size == 64));
+  return (d == 64 || d == 128) && (block_size == 32 || block_size == 64);
 }
 
 cudaError_t launch_fwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const SeqPlan& p,
@@ -325,6 +325,7 @@ cudaError_t launch_fwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v,
     return cudaGetLastError();                                                                                \
   } while (0)
   if (d == 64 && block_size == 32) MOBA_FWD_TC(64, 32);
+  if (d == 64 && block_size == 64) MOBA_FWD_TC(64, 64);
   if (d == 128 && block_size == 32) MOBA_FWD_TC(128, 32);
   if (d == 128 && block_size == 64) MOBA_FWD_TC(128, 64);
 #undef MOBA_FWD_TC

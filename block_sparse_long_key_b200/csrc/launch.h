@@ -72,7 +72,7 @@ cudaError_t launch_fwd_attn(const bf16* q, const bf16* k, const bf16* v, const S
 // the tile::gather4 row gathers).
 cudaError_t make_row_map(CUtensorMap* map, const void* base, unsigned long long nrows, int d, int box_rows = 1);
 
-// tcgen05 forward attention for (d, B) = (64, 32), (128, 32), (128, 64);
+// tcgen05 forward attention for d in {64, 128} and B in {32, 64};
 // `tm_q` is make_row_map over q as T*H_q rows.
 bool fwd_tc_supported(int d, int block_size);
 cudaError_t launch_fwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const SeqPlan& p,
@@ -99,7 +99,7 @@ cudaError_t launch_bwd_attn(const bf16* q, const bf16* k, const bf16* v, const b
                             float* dqacc, bf16* dk, bf16* dv, cudaStream_t st);
 
 // tcgen05 backward attention (dK, dV written; dQ added into dqacc); the
-// shapes it covers (d, B) = (64, 32), (128, 32), (128, 64); tm_q / tm_do are
+// shapes it covers: d in {64, 128}, B in {32, 64}; tm_q / tm_do are
 // make_row_map over q and dout as T*H_q rows.
 bool bwd_tc_supported(int d, int block_size);
 cudaError_t launch_bwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const CUtensorMap& tm_do,
