@@ -49,8 +49,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Headline workload, one timed-step launch each (profiles/dram_traffic_n64k_h16_d64_b32_k32_kconv4.md).
 NCU_TRAFFIC = {
     "fwd_route": {"bytes": 278.41e6 + 366.40e6, "sha": "41a06d3978d3dcd1"},
-    "fwd_attn": {"bytes": 1.1735e9 + 720.60e6, "sha": "87cebeb37e249bda"},
-    "bwd_attn": {"bytes": 1.9499e9 + 1.0257e9, "sha": "fd77383753980c5b"},
+    "fwd_attn": {"bytes": 1.1695e9 + 722.40e6, "sha": "4c84aea0e6808372"},
+    "bwd_attn": {"bytes": 1.9538e9 + 1.0273e9, "sha": "fb01b862248ff62e"},
     "conv_bwd": {"bytes": 268.46e6 + 126.76e6, "sha": "2e8a64640582a328"},
     "fwd_centroid": {"bytes": 134.25e6 + 102.10e6, "sha": "103ae9898d36c11f"},
 }
