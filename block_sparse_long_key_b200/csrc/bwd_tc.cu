@@ -27,10 +27,14 @@
 //      through the free P / dS tiles so that 8 lanes cover one 128-byte row
 //      piece per instruction.
 // The CTA is sequential; a small footprint (one gather stage, 128 TMEM
-// columns at d = 64) lets four CTAs share an SM so that their phases
-// overlap.  At the end dK_j and dV_j are written once (bf16).  Every
-// mbarrier wait is bounded; a timeout sets MOBA_STATUS_TIMEOUT and the CTA
-// winds down.
+// columns at d = 64, B = 32) lets three CTAs share an SM so that their phases
+// overlap.  K_j and V_j arrive once by TMA tile loads (a partial last
+// block's tail rows are zeroed in shared memory).  Block sizes 16 .. 128: the
+// P and dS tiles use the 32-, 64- or 128-byte swizzle (two 128-byte regions
+// at B = 128, where S, dP, dV^T and dK^T take all 512 TMEM columns and one
+// CTA runs per SM).  At the end dK_j and dV_j are written once (bf16).
+// Every mbarrier wait is bounded; a timeout sets MOBA_STATUS_TIMEOUT and the
+// CTA winds down.
 #include "common.cuh"
 #include "launch.h"
 #include "tc.cuh"
@@ -43,22 +47,23 @@ constexpr int kThreads = 128;
 
 template <int D, int BLK>
 struct BwdTcLayout {
+  using PT = tc::KeyTile<BLK>;
   static constexpr int KB = D / 64;                          // 64-wide d chunks (128-byte rows)
   static constexpr uint32_t KV_REGION = BLK * 128;           // one d chunk of K_j or V_j
   static constexpr uint32_t QO_REGION = kRows * 128;         // one d chunk of a Q or dO tile
-  static constexpr uint32_t PROW = BLK * 2;                  // bytes per row of the P / dS tiles
-  static constexpr uint32_t P_BYTES = kRows * PROW;
-  static constexpr uint32_t P_ATOM = BLK == 32 ? 512 : 1024;  // bytes per 8-row group of P / dS
-  static constexpr uint32_t P_LAYOUT = BLK == 32 ? tc::kLayoutSW64 : tc::kLayoutSW128;
   static constexpr uint32_t K_OFF = 0;
   static constexpr uint32_t V_OFF = K_OFF + KB * KV_REGION;
   static constexpr uint32_t P_OFF = V_OFF + KB * KV_REGION;
-  static constexpr uint32_t DS_OFF = P_OFF + P_BYTES;
-  static constexpr uint32_t Q_OFF = DS_OFF + P_BYTES;
+  static constexpr uint32_t DS_OFF = P_OFF + PT::BYTES;
+  // P and dS together, grown to 16 KB where smaller: the dQ rows are staged
+  // there (32 rows x 128 bytes per warp) once the MMAs have read them.
+  static constexpr uint32_t PD_AREA = 2 * PT::BYTES < 16384 ? 16384 : 2 * PT::BYTES;
+  static constexpr uint32_t Q_OFF = P_OFF + PD_AREA;
   static constexpr uint32_t O_OFF = Q_OFF + KB * QO_REGION;
-  static constexpr uint32_t MB_OFF = O_OFF + KB * QO_REGION;  // mbS, mbG, mbQ
-  static constexpr uint32_t HOLD_OFF = MB_OFF + 24;
+  static constexpr uint32_t MB_OFF = O_OFF + KB * QO_REGION;  // mbS, mbG, mbQ, mbKV
+  static constexpr uint32_t HOLD_OFF = MB_OFF + 32;
   static constexpr uint32_t BYTES = HOLD_OFF + 16;
+  static constexpr uint32_t KV_TX = 2 * KB * KV_REGION;      // bytes of one K_j + V_j load
   // Tensor memory columns: S and dP side by side, later overwritten by dQ
   // (D columns); then dV^T and dK^T (B each).
   static constexpr uint32_t S_COL = 0, DP_COL = BLK, DQ_COL = 0;
@@ -66,32 +71,28 @@ struct BwdTcLayout {
   static constexpr uint32_t NCOLS = DK_COL + BLK;
   static constexpr uint32_t TMEM_COLS = NCOLS <= 128 ? 128 : (NCOLS <= 256 ? 256 : 512);
   static_assert(NCOLS <= 512, "tensor memory");
-  static_assert(KV_REGION % 1024 == 0 && P_BYTES % 1024 == 0 && QO_REGION % 1024 == 0,
+  static_assert(KV_REGION % 1024 == 0 && PT::REGION % 1024 == 0 && QO_REGION % 1024 == 0,
                 "swizzle atoms stay aligned");
 };
 
-// Byte offset of the 16-byte chunk c of row r in a P / dS tile.
-template <int BLK>
-__device__ __forceinline__ uint32_t p_offset(int r, int c) {
-  if constexpr (BLK == 32) return tc::sw64_offset(r, c);
-  else return tc::sw128_offset(r, c);
-}
-
 template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads)
-bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__ k, const bf16* __restrict__ v,
-              const __grid_constant__ CUtensorMap tm_do, const float2* __restrict__ stat,
-              const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch, int nb_max,
-              int h_q, int h_kv, int lead, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
-              float* __restrict__ dqacc, bf16* __restrict__ dk, bf16* __restrict__ dv,
-              int32_t* __restrict__ status) {
+bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+              const float2* __restrict__ stat, const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off,
+              int batch, int nb_max, int h_q, int h_kv, int lead, const int32_t* __restrict__ ptr,
+              const int32_t* __restrict__ rows, float* __restrict__ dqacc, bf16* __restrict__ dk,
+              bf16* __restrict__ dv, int32_t* __restrict__ status) {
   using Ly = BwdTcLayout<D, BLK>;
+  using PT = typename Ly::PT;
+  constexpr int CW = BLK < 32 ? BLK : 32;  // TMEM columns per load
   extern __shared__ unsigned char smem_raw[];
   // 1024-byte aligned base, derived from the shared array by pointer
   // arithmetic so that accesses through it stay shared-memory accesses.
   unsigned char* sm = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
   const uint32_t sbase = smem_u32(sm);
-  const uint32_t mb_s = sbase + Ly::MB_OFF, mb_g = mb_s + 8, mb_q = mb_s + 16;
+  const uint32_t mb_s = sbase + Ly::MB_OFF, mb_g = mb_s + 8, mb_q = mb_s + 16, mb_kv = mb_s + 24;
+  mark_path(status, kPathBwdTc);
 
   const BucketOrder bo = bucket_order(blockIdx.x, nb_max, h_kv, lead);
   const int gb = bo.gb, kvh = bo.kvh;
@@ -106,16 +107,6 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
   const float scale = rsqrtf((float)D);
   const float scale_log2 = kLog2e * scale;
   const int ntiles = (end - beg + kRows - 1) / kRows;
-
-  // ---- K_j, V_j -> SW128 K-major (row = key, 64-wide d chunks as regions)
-  for (int i = tid; i < BLK * (D / 8); i += kThreads) {
-    const int r = i / (D / 8), c = i % (D / 8);
-    const bool ok = t0 + r < t1;
-    const size_t off = ok ? (size_t)(t0 + r) * kv_stride + (size_t)kvh * D + c * 8 : 0;
-    const uint32_t o = (c >> 3) * Ly::KV_REGION + tc::sw128_offset(r, c & 7);
-    cp_async16_zfill(sm + Ly::K_OFF + o, k + off, ok);
-    cp_async16_zfill(sm + Ly::V_OFF + o, v + off, ok);
-  }
 
   // Gather this warp's 32 rows of a tile with the TMA: lanes 0..7 each
   // issue one gather4 per 64-wide d chunk and tensor for rows 4l .. 4l+3
@@ -153,10 +144,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
     tc::mbar_init(mb_s, 1);
     tc::mbar_init(mb_g, 1);
     tc::mbar_init(mb_q, kThreads / 32);
+    tc::mbar_init(mb_kv, 1);
     tc::mbar_init_fence();
   }
   if (warp == 0) tc::tmem_alloc(sbase + Ly::HOLD_OFF, Ly::TMEM_COLS);
-  cp_async_commit();
   int rid = meta_rid(0), nrid = -1;
   const float2 st0 = rid >= 0 ? __ldg(stat + rid) : make_float2(0.f, 0.f);  // (LSE, D) of the row
   float lse_c = st0.x, dsum_c = st0.y;
@@ -164,6 +155,16 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  // K_j, V_j -> SW128 K-major tiles (row = key, 64-wide d chunks as
+  // regions): one TMA box of 64 channels x BLK tokens per chunk and tensor.
+  if (ntiles > 0 && tid == 0) {
+    tc::mbar_arrive_expect_tx(mb_kv, Ly::KV_TX);
+#pragma unroll
+    for (int c = 0; c < Ly::KB; ++c) {
+      tc::tma_load_3d(sbase + Ly::K_OFF + c * Ly::KV_REGION, &tm_k, c * 64, kvh, t0, mb_kv);
+      tc::tma_load_3d(sbase + Ly::V_OFF + c * Ly::KV_REGION, &tm_v, c * 64, kvh, t0, mb_kv);
+    }
+  }
   if (ntiles > 0) gather(rid);
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -172,14 +173,24 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
   constexpr uint32_t id_s = tc::idesc_bf16_f32_major(kRows, BLK, 0, 0);  // S, dP
   constexpr uint32_t id_g = tc::idesc_bf16_f32_major(D, BLK, 1, 1);      // dV^T, dK^T
   constexpr uint32_t id_q = tc::idesc_bf16_f32_major(kRows, D, 0, 1);    // dQ
+  // P / dS as the MN-major B operand of dV^T, dK^T: distance between the
+  // 64-key groups (two at B = 128; one otherwise, where it is unused).
+  constexpr uint32_t kPdLbo = PT::NREG > 1 ? PT::REGION : 16;
 
+  // K_j / V_j have landed (decided block-wide); a partial block's tail rows
+  // are cleared, ordered before the first MMA by the barrier of step A.
   bool ok = true;
+  if (ntiles > 0) {
+    ok = __syncthreads_and(tc::mbar_wait(mb_kv, 0));
+    if (ok && t1 - t0 < BLK) {
+      tc::zero_kv_tail_rows<D, BLK>(sm + Ly::K_OFF, sm + Ly::V_OFF, t1 - t0, tid, kThreads);
+      tc::fence_proxy_async();
+    }
+  }
   int it = 0;
-  for (; it < ntiles; ++it) {
+  for (; ok && it < ntiles; ++it) {
     nrid = meta_rid(it + 1);  // consumed by the gather at the end of this tile
-    // A. this tile's rows (and, the first time, K_j / V_j) have landed
-    cp_async_wait<0>();
-    tc::fence_proxy_async();
+    // A. this tile's rows have landed
     const bool landed = tc::mbar_wait(mb_q, it & 1);
     tc::fence_before_sync();
     if (!__syncthreads_and(landed)) {
@@ -210,18 +221,23 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
       const int tok = rid >= 0 ? rid / h_q : -1;
       const float lse2 = lse_c * kLog2e, dsm = dsum_c;
 #pragma unroll
-      for (int h = 0; h < BLK / 32; ++h) {
-        uint32_t sv[32], pv[32];
-        tc::tmem_ld32(tmem + lane_base + Ly::S_COL + h * 32, sv);
-        tc::tmem_ld32(tmem + lane_base + Ly::DP_COL + h * 32, pv);
+      for (int h = 0; h < BLK / CW; ++h) {
+        uint32_t sv[CW], pv[CW];
+        if constexpr (CW == 32) {
+          tc::tmem_ld32(tmem + lane_base + Ly::S_COL + h * CW, *reinterpret_cast<uint32_t(*)[32]>(sv));
+          tc::tmem_ld32(tmem + lane_base + Ly::DP_COL + h * CW, *reinterpret_cast<uint32_t(*)[32]>(pv));
+        } else {
+          tc::tmem_ld16(tmem + lane_base + Ly::S_COL + h * CW, sv);
+          tc::tmem_ld16(tmem + lane_base + Ly::DP_COL + h * CW, pv);
+        }
         tc::tmem_ld_wait();
-        uint32_t pp[16], dd[16];
+        uint32_t pp[CW / 2], dd[CW / 2];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
+        for (int c = 0; c < CW; c += 2) {
           float p2[2], d2[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int key_tok = t0 + h * 32 + c + u;
+            const int key_tok = t0 + h * CW + c + u;
             float p = 0.f;
             if (key_tok <= tok && key_tok < t1) p = fast_exp2(__uint_as_float(sv[c + u]) * scale_log2 - lse2);
             p2[u] = p;
@@ -231,8 +247,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
           dd[c / 2] = pack_bf16(d2[0], d2[1]);
         }
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t o = p_offset<BLK>(tid, h * 4 + c);
+        for (int c = 0; c < CW / 8; ++c) {
+          const uint32_t o = PT::offset(tid, h * (CW / 8) + c);
           *reinterpret_cast<uint4*>(sm + Ly::P_OFF + o) =
               make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
           *reinterpret_cast<uint4*>(sm + Ly::DS_OFF + o) =
@@ -255,17 +271,18 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
       for (int ks = 0; ks < kRows / 16; ++ks) {
         // 16 rows = two 8-row groups of the Q / dO tiles and of P / dS
         const uint32_t ro = ks * 2048;
-        const uint32_t po = ks * 2 * Ly::P_ATOM;
+        const uint32_t po = ks * 2 * PT::ATOM;
         const uint32_t acc = (it > 0 || ks > 0) ? 1u : 0u;
         tc::mma_bf16_ss(tmem + Ly::DV_COL, tc::smem_desc(oa + ro, Ly::QO_REGION, 1024, tc::kLayoutSW128),
-                        tc::smem_desc(sbase + Ly::P_OFF + po, 16, Ly::P_ATOM, Ly::P_LAYOUT), id_g, acc);
+                        tc::smem_desc(sbase + Ly::P_OFF + po, kPdLbo, PT::ATOM, PT::LAYOUT), id_g, acc);
         tc::mma_bf16_ss(tmem + Ly::DK_COL, tc::smem_desc(qa + ro, Ly::QO_REGION, 1024, tc::kLayoutSW128),
-                        tc::smem_desc(sbase + Ly::DS_OFF + po, 16, Ly::P_ATOM, Ly::P_LAYOUT), id_g, acc);
+                        tc::smem_desc(sbase + Ly::DS_OFF + po, kPdLbo, PT::ATOM, PT::LAYOUT), id_g, acc);
       }
 #pragma unroll
       for (int kk = 0; kk < BLK / 16; ++kk) {
         // K steps of 16 keys: 32 bytes along a dS row; two 8-key groups of K_j
-        tc::mma_bf16_ss(tmem + Ly::DQ_COL, tc::smem_desc(sbase + Ly::DS_OFF + kk * 32, 16, Ly::P_ATOM, Ly::P_LAYOUT),
+        const uint32_t po = (uint32_t)((kk * 32) / PT::ROWB) * PT::REGION + (uint32_t)((kk * 32) % PT::ROWB);
+        tc::mma_bf16_ss(tmem + Ly::DQ_COL, tc::smem_desc(sbase + Ly::DS_OFF + po, 16, PT::ATOM, PT::LAYOUT),
                         tc::smem_desc(sbase + Ly::K_OFF + kk * 2048, Ly::KV_REGION, 1024, tc::kLayoutSW128), id_q,
                         kk > 0);
       }
@@ -279,7 +296,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
     }
     tc::fence_after_sync();
     if (it + 1 < ntiles) gather(nrid);
-    // dQ rows leave through the (now free) P / dS tiles: each warp stages
+    // dQ rows leave through the (now free) P / dS area: each warp stages
     // 32-column halves of its 32 rows, then 8 lanes cover one 128-byte row
     // piece per reduction instruction.
     unsigned char* stg = sm + Ly::P_OFF + warp * 4096;
@@ -309,16 +326,17 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
     dsum_c = dsum_n;
   }
   const int fail_it = it;
-  cp_async_wait<0>();
   tc::fence_before_sync();
-  __syncthreads();
+  ok = __syncthreads_and(ok);
   if (!ok) {
-    // A tensor-core completion never arrived: record it, give the MMAs in
-    // flight a bounded chance to drain, release TMEM, leave dK_j / dV_j alone.
+    // A tensor-core or TMA completion never arrived: record it, give the
+    // MMAs and copies in flight a bounded chance to drain (a wait on a phase
+    // that is not pending returns at once), release TMEM, leave dK_j / dV_j
+    // alone.
     if (tid == 0) set_status(status, kStatusTimeout);
+    tc::mbar_wait(mb_kv, 0, 100000000ull);
     tc::mbar_wait(mb_s, fail_it & 1, 100000000ull);
     tc::mbar_wait(mb_g, fail_it & 1, 100000000ull);
-    // a gather in flight (this tile's or the next) lands before exit
     tc::mbar_wait(mb_q, fail_it & 1, 100000000ull);
     tc::mbar_wait(mb_q, (fail_it + 1) & 1, 100000000ull);
     __syncthreads();
@@ -330,15 +348,20 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
   // in lane (m % 16) + 32 (m / 16) for M = 64.
   const int m = D == 128 ? tid : (lane < 16 ? warp * 16 + lane : -1);
 #pragma unroll
-  for (int h = 0; h < BLK / 32; ++h) {
-    uint32_t av[32], bv[32];
-    tc::tmem_ld32(tmem + lane_base + Ly::DV_COL + h * 32, av);
-    tc::tmem_ld32(tmem + lane_base + Ly::DK_COL + h * 32, bv);
+  for (int h = 0; h < BLK / CW; ++h) {
+    uint32_t av[CW], bv[CW];
+    if constexpr (CW == 32) {
+      tc::tmem_ld32(tmem + lane_base + Ly::DV_COL + h * CW, *reinterpret_cast<uint32_t(*)[32]>(av));
+      tc::tmem_ld32(tmem + lane_base + Ly::DK_COL + h * CW, *reinterpret_cast<uint32_t(*)[32]>(bv));
+    } else {
+      tc::tmem_ld16(tmem + lane_base + Ly::DV_COL + h * CW, av);
+      tc::tmem_ld16(tmem + lane_base + Ly::DK_COL + h * CW, bv);
+    }
     tc::tmem_ld_wait();
     if (m >= 0) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int kt = t0 + h * 32 + c;
+      for (int c = 0; c < CW; ++c) {
+        const int kt = t0 + h * CW + c;
         const float a = ntiles > 0 ? __uint_as_float(av[c]) : 0.f;
         const float b = ntiles > 0 ? __uint_as_float(bv[c]) * scale : 0.f;
         if (kt < t1) {
@@ -356,12 +379,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
 
 }  // namespace
 
-bool bwd_tc_supported(int d, int block_size) {
-  return (d == 64 || d == 128) && (block_size == 32 || block_size == 64);
-}
-
-cudaError_t launch_bwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const CUtensorMap& tm_do,
-                          const float2* stat, const SeqPlan& p, const int32_t* ptr,
+cudaError_t launch_bwd_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                          const CUtensorMap& tm_do, const float2* stat, const SeqPlan& p, const int32_t* ptr,
                           const int32_t* rows, int h_q, int h_kv, int d, int block_size, float* dqacc, bf16* dk,
                           bf16* dv, int32_t* status, cudaStream_t st) {
 #define MOBA_BWD_TC(DD, BB)                                                                                  \
@@ -372,15 +391,21 @@ cudaError_t launch_bwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v,
     if (e != cudaSuccess) return e;                                                                          \
     if (p.nb_max == 0) return cudaSuccess;                                                                   \
     const int lead = bucket_lead((long long)p.total_tokens * (h_q / h_kv), DD * 4);                          \
-    kern<<<dim3(p.nb_max * h_kv), kThreads, smem, st>>>(tm_q, k, v, tm_do, stat, p.cu, p.blk_off, p.batch, \
-                                                       p.nb_max, h_q, h_kv, lead, ptr, rows, dqacc, dk, dv,   \
-                                                       status);                                                \
+    kern<<<dim3(p.nb_max * h_kv), kThreads, smem, st>>>(tm_q, tm_k, tm_v, tm_do, stat, p.cu, p.blk_off,     \
+                                                       p.batch, p.nb_max, h_q, h_kv, lead, ptr, rows, dqacc, \
+                                                       dk, dv, status);                                      \
     return cudaGetLastError();                                                                               \
   } while (0)
-  if (d == 64 && block_size == 32) MOBA_BWD_TC(64, 32);
-  if (d == 64 && block_size == 64) MOBA_BWD_TC(64, 64);
-  if (d == 128 && block_size == 32) MOBA_BWD_TC(128, 32);
-  if (d == 128 && block_size == 64) MOBA_BWD_TC(128, 64);
+#define MOBA_BWD_TC_B(DD)           \
+  switch (block_size) {             \
+    case 16: MOBA_BWD_TC(DD, 16);   \
+    case 32: MOBA_BWD_TC(DD, 32);   \
+    case 64: MOBA_BWD_TC(DD, 64);   \
+    case 128: MOBA_BWD_TC(DD, 128); \
+  }
+  if (d == 64) MOBA_BWD_TC_B(64);
+  if (d == 128) MOBA_BWD_TC_B(128);
+#undef MOBA_BWD_TC_B
 #undef MOBA_BWD_TC
   return cudaErrorInvalidValue;
 }

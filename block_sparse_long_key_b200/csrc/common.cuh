@@ -20,6 +20,20 @@ __device__ __forceinline__ void set_status(int32_t* status, int32_t bit) {
   atomicOr(reinterpret_cast<int*>(status), bit);
 }
 
+// Kernel-path bits, OR-ed into the word after the status word (status[1])
+// and reported by moba_check_path(): which kernel families ran.
+enum : int32_t {
+  kPathRouteTc = 1 << 0,    // route_kernel (tcgen05 scores)
+  kPathFwdTc = 1 << 1,      // fwd_tc_kernel (tcgen05 forward attention)
+  kPathBwdTc = 1 << 2,      // bwd_tc_kernel (tcgen05 backward attention)
+  kPathExactRows = 1 << 3   // fwd_fallback_kernel recomputed at least one row
+};
+
+// Marks that the calling kernel ran: one atomic from the grid's first thread.
+__device__ __forceinline__ void mark_path(int32_t* status, int32_t bit) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(reinterpret_cast<int*>(status + 1), bit);
+}
+
 // Largest s with off[s] <= x, for off[0..n] non-decreasing, off[0] <= x.
 __device__ __forceinline__ int upper_seq(const int32_t* off, int n, int x) {
   int lo = 0, hi = n;  // answer in [0, n)

@@ -7,7 +7,10 @@
 // block, scatter the results).
 //
 // One CTA per (global key block j, KV head) walks the block's bucket in
-// tiles of 128 gathered rows; thread t owns tile row t = TMEM lane t.
+// tiles of 128 gathered rows; thread t owns tile row t = TMEM lane t.  K_j
+// and V_j arrive once, by TMA tile loads (64 channels x B tokens per box,
+// 128-byte swizzle); rows of a partial last block are zeroed in shared
+// memory before use.
 //   1. Q rows are gathered by the TMA (tile::gather4, four rows per
 //      instruction, 128-byte swizzle) into a K-major tile; completion is
 //      counted in bytes on an mbarrier.
@@ -24,9 +27,11 @@
 //      16-byte vector reduction into the query's fp32 accumulator row (d
 //      floats), so an instruction touches 4 rows, not 16 (one line each).
 // The merge of a query's k blocks is therefore a plain sum; finalize divides
-// by l.  A CTA needs ~41 KB of shared memory and 64 TMEM columns at d = 64,
-// so five share an SM and overlap their phases.  Every mbarrier wait is
-// bounded; a timeout sets MOBA_STATUS_TIMEOUT and the CTA winds down.
+// by l.  Block sizes 16 .. 128: the P tile uses the 32-, 64- or 128-byte
+// swizzle (two 128-byte regions at B = 128).  A CTA needs ~41 KB of shared
+// memory and 64 TMEM columns at d = 64, B = 32, so five share an SM and
+// overlap their phases.  Every mbarrier wait is bounded; a timeout sets
+// MOBA_STATUS_TIMEOUT and the CTA winds down.
 #include "common.cuh"
 #include "launch.h"
 #include "tc.cuh"
@@ -40,51 +45,48 @@ constexpr float kOverflowLog2 = 90.f;  // ~62 in natural-log units
 
 template <int D, int BLK>
 struct FwdTcLayout {
+  using PT = tc::KeyTile<BLK>;
   static constexpr int KB = D / 64;                          // 64-wide d chunks (128-byte rows)
   static constexpr uint32_t KV_REGION = BLK * 128;           // one d chunk of K_j or V_j
   static constexpr uint32_t Q_REGION = kRows * 128;          // one d chunk of the Q tile
-  static constexpr uint32_t PROW = BLK * 2;                  // bytes per P row
-  static constexpr uint32_t P_BYTES = kRows * PROW;
-  static constexpr uint32_t P_ATOM = BLK == 32 ? 512 : 1024;  // bytes per 8-row group of P
-  static constexpr uint32_t P_LAYOUT = BLK == 32 ? tc::kLayoutSW64 : tc::kLayoutSW128;
   static constexpr uint32_t K_OFF = 0;
   static constexpr uint32_t V_OFF = K_OFF + KB * KV_REGION;
   static constexpr uint32_t Q_OFF = V_OFF + KB * KV_REGION;
   static constexpr uint32_t P_OFF = Q_OFF + KB * Q_REGION;
   // The P tile, grown to 16 KB where it is smaller, doubles as the staging
-  // area of the O reductions (32 rows x 128 bytes per warp).
-  static constexpr uint32_t STG_BYTES = P_BYTES < 16384 ? 16384 : P_BYTES;
-  static constexpr uint32_t MB_OFF = P_OFF + STG_BYTES;    // mbS, mbO, mbQ
-  static constexpr uint32_t HOLD_OFF = MB_OFF + 24;
+  // area of the O reductions (its first 16 KB: 32 rows x 128 bytes per warp).
+  static constexpr uint32_t STG_BYTES = 16384;
+  static constexpr uint32_t P_AREA = PT::BYTES < STG_BYTES ? STG_BYTES : PT::BYTES;
+  static constexpr uint32_t MB_OFF = P_OFF + P_AREA;    // mbS, mbO, mbQ, mbKV
+  static constexpr uint32_t HOLD_OFF = MB_OFF + 32;
   static constexpr uint32_t BYTES = HOLD_OFF + 16;
+  static constexpr uint32_t KV_TX = 2 * KB * KV_REGION;      // bytes of one K_j + V_j load
   // Tensor memory: S (B columns), later overwritten by O (D columns).
   static constexpr uint32_t NCOLS = BLK > D ? BLK : D;
   static constexpr uint32_t TMEM_COLS = NCOLS <= 32 ? 32 : (NCOLS <= 64 ? 64 : (NCOLS <= 128 ? 128 : 256));
-  static_assert(KV_REGION % 1024 == 0 && P_BYTES % 1024 == 0 && Q_REGION % 1024 == 0, "swizzle atoms stay aligned");
+  static_assert(KV_REGION % 1024 == 0 && PT::REGION % 1024 == 0 && Q_REGION % 1024 == 0,
+                "swizzle atoms stay aligned");
 };
-
-template <int BLK>
-__device__ __forceinline__ uint32_t p_offset(int r, int c) {
-  if constexpr (BLK == 32) return tc::sw64_offset(r, c);
-  else return tc::sw128_offset(r, c);
-}
 
 template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads)
-fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__ k, const bf16* __restrict__ v,
-              const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch, int nb_max,
-              int h_q, int h_kv, int lead, const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows,
-              const float* __restrict__ mref, float* __restrict__ oacc, float* __restrict__ lacc,
-              int32_t* __restrict__ flag,
+fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ cu,
+              const int32_t* __restrict__ blk_off, int batch, int nb_max, int h_q, int h_kv, int lead,
+              const int32_t* __restrict__ ptr, const int32_t* __restrict__ rows, const float* __restrict__ mref,
+              float* __restrict__ oacc, float* __restrict__ lacc, int32_t* __restrict__ flag,
               int32_t* __restrict__ status) {
   using Ly = FwdTcLayout<D, BLK>;
+  using PT = typename Ly::PT;
   constexpr int OS = oacc_stride(D);
+  constexpr int CW = BLK < 32 ? BLK : 32;  // S columns per TMEM load
   extern __shared__ unsigned char smem_raw[];
   // 1024-byte aligned base, derived from the shared array by pointer
   // arithmetic so that accesses through it stay shared-memory accesses.
   unsigned char* sm = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
   const uint32_t sbase = smem_u32(sm);
-  const uint32_t mb_s = sbase + Ly::MB_OFF, mb_o = mb_s + 8, mb_q = mb_s + 16;
+  const uint32_t mb_s = sbase + Ly::MB_OFF, mb_o = mb_s + 8, mb_q = mb_s + 16, mb_kv = mb_s + 24;
+  mark_path(status, kPathFwdTc);
 
   const BucketOrder bo = bucket_order(blockIdx.x, nb_max, h_kv, lead);
   const int gb = bo.gb, kvh = bo.kvh;
@@ -96,19 +98,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
   const int t0 = __ldg(cu + s) + (gb - __ldg(blk_off + s)) * BLK;
   const int t1 = min(t0 + BLK, __ldg(cu + s + 1));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const size_t kv_stride = (size_t)h_kv * D;
   const float scale_log2 = kLog2e * rsqrtf((float)D);
   const int ntiles = (end - beg + kRows - 1) / kRows;
 
-  // ---- K_j, V_j -> SW128 K-major (row = key, 64-wide d chunks as regions)
-  for (int i = tid; i < BLK * (D / 8); i += kThreads) {
-    const int r = i / (D / 8), c = i % (D / 8);
-    const bool ok = t0 + r < t1;
-    const size_t off = ok ? (size_t)(t0 + r) * kv_stride + (size_t)kvh * D + c * 8 : 0;
-    const uint32_t o = (c >> 3) * Ly::KV_REGION + tc::sw128_offset(r, c & 7);
-    cp_async16_zfill(sm + Ly::K_OFF + o, k + off, ok);
-    cp_async16_zfill(sm + Ly::V_OFF + o, v + off, ok);
-  }
   // Gather this warp's 32 rows of a tile with the TMA: lanes 0..7 each
   // issue one gather4 per 64-wide d chunk for rows 4l .. 4l+3 (row ids from
   // the lanes' `r_`; a missing row reads row 0, whose P is zero).
@@ -137,15 +129,25 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
     tc::mbar_init(mb_s, 1);
     tc::mbar_init(mb_o, 1);
     tc::mbar_init(mb_q, kThreads / 32);
+    tc::mbar_init(mb_kv, 1);
     tc::mbar_init_fence();
   }
   if (warp == 0) tc::tmem_alloc(sbase + Ly::HOLD_OFF, Ly::TMEM_COLS);
-  cp_async_commit();
   int rid = meta_rid(0), nrid = -1;
   float mr_c = rid >= 0 ? __ldg(mref + rid) * kLog2e : 0.f, mr_n = 0.f;
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  // K_j, V_j -> SW128 K-major tiles (row = key, 64-wide d chunks as
+  // regions): one TMA box of 64 channels x BLK tokens per chunk and tensor.
+  if (tid == 0) {
+    tc::mbar_arrive_expect_tx(mb_kv, Ly::KV_TX);
+#pragma unroll
+    for (int c = 0; c < Ly::KB; ++c) {
+      tc::tma_load_3d(sbase + Ly::K_OFF + c * Ly::KV_REGION, &tm_k, c * 64, kvh, t0, mb_kv);
+      tc::tma_load_3d(sbase + Ly::V_OFF + c * Ly::KV_REGION, &tm_v, c * 64, kvh, t0, mb_kv);
+    }
+  }
   gather(rid);
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -153,13 +155,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
   constexpr uint32_t id_s = tc::idesc_bf16_f32_major(kRows, BLK, 0, 0);  // S = Q K^T
   constexpr uint32_t id_o = tc::idesc_bf16_f32_major(kRows, D, 0, 1);    // O = P V
 
-  bool ok = true;
-  int it = 0;
-  for (; it < ntiles; ++it) {
-    nrid = meta_rid(it + 1);
-    // A. this tile's rows (and, the first time, K_j / V_j) have landed
-    cp_async_wait<0>();
+  // K_j / V_j have landed (decided block-wide); a partial block's tail rows
+  // are cleared, ordered before the first MMA by the barrier of step A.
+  bool ok = __syncthreads_and(tc::mbar_wait(mb_kv, 0));
+  if (ok && t1 - t0 < BLK) {
+    tc::zero_kv_tail_rows<D, BLK>(sm + Ly::K_OFF, sm + Ly::V_OFF, t1 - t0, tid, kThreads);
     tc::fence_proxy_async();
+  }
+  int it = 0;
+  for (; ok && it < ntiles; ++it) {
+    nrid = meta_rid(it + 1);
+    // A. this tile's rows have landed
     const bool landed = tc::mbar_wait(mb_q, it & 1);
     tc::fence_before_sync();
     if (!__syncthreads_and(landed)) {
@@ -189,17 +195,18 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
     {
       const int tok = rid >= 0 ? rid / h_q : -1;
 #pragma unroll
-      for (int h = 0; h < BLK / 32; ++h) {
-        uint32_t sv[32];
-        tc::tmem_ld32(tmem + lane_base + h * 32, sv);
+      for (int h = 0; h < BLK / CW; ++h) {
+        uint32_t sv[CW];
+        if constexpr (CW == 32) tc::tmem_ld32(tmem + lane_base + h * CW, *reinterpret_cast<uint32_t(*)[32]>(sv));
+        else tc::tmem_ld16(tmem + lane_base + h * CW, sv);
         tc::tmem_ld_wait();
-        uint32_t pp[16];
+        uint32_t pp[CW / 2];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
+        for (int c = 0; c < CW; c += 2) {
           float p2[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int key_tok = t0 + h * 32 + c + u;
+            const int key_tok = t0 + h * CW + c + u;
             float p = 0.f;
             if (key_tok <= tok && key_tok < t1) {
               const float x = __uint_as_float(sv[c + u]) * scale_log2;
@@ -212,8 +219,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
           pp[c / 2] = pack_bf16(p2[0], p2[1]);
         }
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(sm + Ly::P_OFF + p_offset<BLK>(tid, h * 4 + c)) =
+        for (int c = 0; c < CW / 8; ++c)
+          *reinterpret_cast<uint4*>(sm + Ly::P_OFF + PT::offset(tid, h * (CW / 8) + c)) =
               make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
       }
     }
@@ -221,14 +228,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
-    // D. O = P V_j into the score columns
+    // D. O = P V_j into the score columns (K steps of 16 keys: 32 bytes of a
+    // P row; 16 rows = 2048 bytes of V_j)
     if (tid == 0) {
       tc::fence_after_sync();
 #pragma unroll
-      for (int kk = 0; kk < BLK / 16; ++kk)
-        tc::mma_bf16_ss(tmem, tc::smem_desc(sbase + Ly::P_OFF + kk * 32, 16, Ly::P_ATOM, Ly::P_LAYOUT),
+      for (int kk = 0; kk < BLK / 16; ++kk) {
+        const uint32_t po = (uint32_t)((kk * 32) / PT::ROWB) * PT::REGION + (uint32_t)((kk * 32) % PT::ROWB);
+        tc::mma_bf16_ss(tmem, tc::smem_desc(sbase + Ly::P_OFF + po, 16, PT::ATOM, PT::LAYOUT),
                         tc::smem_desc(sbase + Ly::V_OFF + kk * 2048, Ly::KV_REGION, 1024, tc::kLayoutSW128), id_o,
                         kk > 0);
+      }
       tc::mma_commit(mb_o);
     }
     // E. add the O row and l to the accumulator
@@ -241,39 +251,30 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
       atomicAdd(lacc + rid, l);
       if (mx - mr_c > kOverflowLog2) flag[rid] = 1;
     }
-    // O rows leave through the (now free) P tile: each warp stages CPP-column
-    // pieces of its 32 rows, then LPR lanes cover one row piece per 16-byte
-    // reduction (fewer rows per instruction than one lane per row).
+    // O rows leave through the (now free) P tile: each warp stages 32-column
+    // pieces of its 32 rows, then 8 lanes cover one 128-byte row piece per
+    // 16-byte reduction (4 rows per instruction instead of one per lane).
     {
-      constexpr int CPP = (int)(Ly::STG_BYTES / 4) / (32 * 4);  // columns per pass
-      constexpr int RB = CPP * 4;                              // bytes per staged row piece
-      constexpr int LPR = RB / 16;                             // lanes per row piece
-      constexpr int RPI = 32 / LPR;                            // rows per instruction
-      static_assert(32 % CPP == 0 && LPR >= 4, "staging geometry");
-      unsigned char* stg = sm + Ly::P_OFF + warp * (32 * RB);
-      auto swz = [](int row, int c) { return LPR == 8 ? (c ^ (row & 7)) : (c ^ ((row >> 1) & 3)); };
+      unsigned char* stg = sm + Ly::P_OFF + warp * 4096;
 #pragma unroll
       for (int h = 0; h < D / 32; ++h) {
         uint32_t ov[32];
         tc::tmem_ld32(tmem + lane_base + h * 32, ov);
         tc::tmem_ld_wait();
 #pragma unroll
-        for (int ps = 0; ps < 32 / CPP; ++ps) {
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<float4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+              make_float4(__uint_as_float(ov[4 * c]), __uint_as_float(ov[4 * c + 1]),
+                          __uint_as_float(ov[4 * c + 2]), __uint_as_float(ov[4 * c + 3]));
+        __syncwarp();
 #pragma unroll
-          for (int c = 0; c < LPR; ++c)
-            *reinterpret_cast<float4*>(stg + lane * RB + (swz(lane, c) << 4)) =
-                make_float4(__uint_as_float(ov[ps * CPP + 4 * c]), __uint_as_float(ov[ps * CPP + 4 * c + 1]),
-                            __uint_as_float(ov[ps * CPP + 4 * c + 2]), __uint_as_float(ov[ps * CPP + 4 * c + 3]));
-          __syncwarp();
-#pragma unroll
-          for (int i = 0; i < 32 / RPI; ++i) {
-            const int rl = i * RPI + lane / LPR, c = lane % LPR;
-            const float4 val = *reinterpret_cast<const float4*>(stg + rl * RB + (swz(rl, c) << 4));
-            const int row = __shfl_sync(0xffffffffu, rid, rl);
-            if (row >= 0) red_add_v4(oacc + (size_t)row * OS + h * 32 + ps * CPP + c * 4, val.x, val.y, val.z, val.w);
-          }
-          __syncwarp();
+        for (int i = 0; i < 8; ++i) {
+          const int rl = i * 4 + (lane >> 3), c = lane & 7;
+          const float4 val = *reinterpret_cast<const float4*>(stg + rl * 128 + ((c ^ (rl & 7)) << 4));
+          const int row = __shfl_sync(0xffffffffu, rid, rl);
+          if (row >= 0) red_add_v4(oacc + (size_t)row * OS + h * 32 + c * 4, val.x, val.y, val.z, val.w);
         }
+        __syncwarp();
       }
     }
     tc::fence_before_sync();
@@ -281,17 +282,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
     mr_c = mr_n;
   }
   const int fail_it = it;
-  cp_async_wait<0>();
   tc::fence_before_sync();
-  __syncthreads();
+  ok = __syncthreads_and(ok);
   if (!ok) {
-    // A tensor-core completion never arrived: record it, give the MMAs in
-    // flight a bounded chance to drain, release TMEM.
+    // A tensor-core or TMA completion never arrived: record it, give the
+    // MMAs and copies in flight a bounded chance to drain (a wait on a phase
+    // that is not pending returns at once), release TMEM.
     if (tid == 0) set_status(status, kStatusTimeout);
+    tc::mbar_wait(mb_kv, 0, 100000000ull);
     tc::mbar_wait(mb_s, fail_it & 1, 100000000ull);
     tc::mbar_wait(mb_o, fail_it & 1, 100000000ull);
-    // A gather in flight (for this tile or the next) lands before exit: the
-    // wait on the phase that is not pending returns at once.
     tc::mbar_wait(mb_q, fail_it & 1, 100000000ull);
     tc::mbar_wait(mb_q, (fail_it + 1) & 1, 100000000ull);
     __syncthreads();
@@ -304,14 +304,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const bf16* __restrict__
 
 }  // namespace
 
-bool fwd_tc_supported(int d, int block_size) {
-  return (d == 64 || d == 128) && (block_size == 32 || block_size == 64);
-}
-
-cudaError_t launch_fwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const SeqPlan& p,
-                          const int32_t* ptr, const int32_t* rows, const float* mref, int h_q, int h_kv, int d,
-                          int block_size, float* oacc, float* lacc, int32_t* flag, int32_t* status,
-                          cudaStream_t st) {
+cudaError_t launch_fwd_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                          const SeqPlan& p, const int32_t* ptr, const int32_t* rows, const float* mref, int h_q,
+                          int h_kv, int d, int block_size, float* oacc, float* lacc, int32_t* flag,
+                          int32_t* status, cudaStream_t st) {
 #define MOBA_FWD_TC(DD, BB)                                                                                   \
   do {                                                                                                        \
     const size_t smem = FwdTcLayout<DD, BB>::BYTES + 1024;                                                    \
@@ -320,14 +316,21 @@ cudaError_t launch_fwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v,
     if (e != cudaSuccess) return e;                                                                           \
     if (p.nb_max == 0) return cudaSuccess;                                                                    \
     const int lead = bucket_lead((long long)p.total_tokens * (h_q / h_kv), DD * 4 + 4);                     \
-    kern<<<dim3(p.nb_max * h_kv), kThreads, smem, st>>>(tm_q, k, v, p.cu, p.blk_off, p.batch, p.nb_max, h_q,   \
-                                                       h_kv, lead, ptr, rows, mref, oacc, lacc, flag, status);      \
+    kern<<<dim3(p.nb_max * h_kv), kThreads, smem, st>>>(tm_q, tm_k, tm_v, p.cu, p.blk_off, p.batch, p.nb_max, \
+                                                       h_q, h_kv, lead, ptr, rows, mref, oacc, lacc, flag,    \
+                                                       status);                                               \
     return cudaGetLastError();                                                                                \
   } while (0)
-  if (d == 64 && block_size == 32) MOBA_FWD_TC(64, 32);
-  if (d == 64 && block_size == 64) MOBA_FWD_TC(64, 64);
-  if (d == 128 && block_size == 32) MOBA_FWD_TC(128, 32);
-  if (d == 128 && block_size == 64) MOBA_FWD_TC(128, 64);
+#define MOBA_FWD_TC_B(DD)                         \
+  switch (block_size) {                           \
+    case 16: MOBA_FWD_TC(DD, 16);                 \
+    case 32: MOBA_FWD_TC(DD, 32);                 \
+    case 64: MOBA_FWD_TC(DD, 64);                 \
+    case 128: MOBA_FWD_TC(DD, 128);               \
+  }
+  if (d == 64) MOBA_FWD_TC_B(64);
+  if (d == 128) MOBA_FWD_TC_B(128);
+#undef MOBA_FWD_TC_B
 #undef MOBA_FWD_TC
   return cudaErrorInvalidValue;
 }

@@ -11,12 +11,13 @@
 // The array is a file-scope __device__ variable: every GPU that loads the
 // library holds MOBA_NOALLOC_SCRATCH_BYTES of it until the process exits.
 // In host code its name is only a host-side handle, not a device address, so
-// the first call on each device looks the address up with
-// cudaGetSymbolAddress (with that device current) and caches it.
+// every call looks the address up with cudaGetSymbolAddress on the current
+// device.  The lookup is a host-side query (no device work, no allocation);
+// re-doing it per call keeps the pointer valid for the context that is
+// current now, also after a cudaDeviceReset re-created it.
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 
 #include "moba.h"
 #include "launch.h"
@@ -25,26 +26,15 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_index_scratch[MOBA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
 constexpr size_t kAlign = 256;
-
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Device address of the scratch array on the current device (looked up once).
+// Device address of the scratch array in the current device's context.
 int scratch_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOBA_ELAUNCH;
-  if (dev < 0 || dev >= kMaxDevices) return MOBA_EINVAL;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_index_scratch) != cudaSuccess || !p) return MOBA_ELAUNCH;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_index_scratch) != cudaSuccess || !p) return MOBA_ELAUNCH;
+  *out = p;
   return MOBA_OK;
 }
 

@@ -62,48 +62,41 @@ cudaError_t launch_build_index(const int32_t* sel_idx, const SeqPlan& p, int h_q
                                int block_size, int topk, int32_t* cnt, int32_t* ptr, int32_t* cursor,
                                int32_t* rows, int32_t* status, cudaStream_t st, int32_t* chunk_cnt = nullptr);
 
-cudaError_t launch_fwd_attn(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p,
-                            const int32_t* ptr, const int32_t* rows, const float* mref, int h_q,
-                            int h_kv, int d, int block_size, float* oacc, float* lacc, int32_t* flag,
-                            cudaStream_t st);
-
 // Tensor map over a [nrows, d] bf16 row table (16-byte aligned base):
 // 64-element boxes `box_rows` rows high, 128-byte swizzle (box_rows = 1 for
 // the tile::gather4 row gathers).
 cudaError_t make_row_map(CUtensorMap* map, const void* base, unsigned long long nrows, int d, int box_rows = 1);
 
-// tcgen05 forward attention for d in {64, 128} and B in {32, 64};
-// `tm_q` is make_row_map over q as T*H_q rows.
-bool fwd_tc_supported(int d, int block_size);
-cudaError_t launch_fwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const SeqPlan& p,
-                          const int32_t* ptr, const int32_t* rows, const float* mref, int h_q, int h_kv, int d,
-                          int block_size, float* oacc, float* lacc, int32_t* flag, int32_t* status,
-                          cudaStream_t st);
+// Tensor map over a [T, h_kv, d] bf16 key or value tensor: boxes of 64
+// channels x one head x `box_tokens` tokens (a key block), 128-byte swizzle.
+cudaError_t make_kv_map(CUtensorMap* map, const void* base, int total_tokens, int h_kv, int d, int box_tokens);
+
+// tcgen05 forward attention (every supported d and B); `tm_q` is
+// make_row_map over q as T*H_q rows, `tm_k` / `tm_v` make_kv_map over k and v
+// with box_tokens = block_size.
+cudaError_t launch_fwd_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                          const SeqPlan& p, const int32_t* ptr, const int32_t* rows, const float* mref, int h_q,
+                          int h_kv, int d, int block_size, float* oacc, float* lacc, int32_t* flag,
+                          int32_t* status, cudaStream_t st);
 
 cudaError_t launch_fwd_finalize(const float* oacc, const float* lacc, const float* mref, const int32_t* flag, int nrows,
                                 int d, bf16* out, float* lse, int32_t* flag_list, cudaStream_t st);
 
 cudaError_t launch_fwd_fallback(const bf16* q, const bf16* k, const bf16* v, const SeqPlan& p,
                                 const int32_t* sel_idx, const int32_t* flag_list, int h_q, int h_kv,
-                                int d, int block_size, int topk, bf16* out, float* lse,
+                                int d, int block_size, int topk, bf16* out, float* lse, int32_t* status,
                                 cudaStream_t st);
 
-// dsum[row] = D_i = dO_i . O_i; stat[row] = (LSE_i, D_i) for the tcgen05
-// backward (one 8-byte load per gathered row); zeroes the dQ accumulator.
-cudaError_t launch_bwd_pre(const bf16* out, const bf16* dout, const float* lse, int nrows, int d, float* dsum,
-                           float2* stat, float* dqacc, cudaStream_t st);
+// stat[row] = (LSE_i, D_i = dO_i . O_i) for the tcgen05 backward (one 8-byte
+// load per gathered row); zeroes the dQ accumulator.
+cudaError_t launch_bwd_pre(const bf16* out, const bf16* dout, const float* lse, int nrows, int d, float2* stat,
+                           float* dqacc, cudaStream_t st);
 
-cudaError_t launch_bwd_attn(const bf16* q, const bf16* k, const bf16* v, const bf16* dout,
-                            const float* lse, const float* dsum, const SeqPlan& p, const int32_t* ptr,
-                            const int32_t* rows, int h_q, int h_kv, int d, int block_size,
-                            float* dqacc, bf16* dk, bf16* dv, cudaStream_t st);
-
-// tcgen05 backward attention (dK, dV written; dQ added into dqacc); the
-// shapes it covers: d in {64, 128}, B in {32, 64}; tm_q / tm_do are
-// make_row_map over q and dout as T*H_q rows.
-bool bwd_tc_supported(int d, int block_size);
-cudaError_t launch_bwd_tc(const CUtensorMap& tm_q, const bf16* k, const bf16* v, const CUtensorMap& tm_do,
-                          const float2* stat, const SeqPlan& p, const int32_t* ptr,
+// tcgen05 backward attention (dK, dV written; dQ added into dqacc) for
+// every supported d and B; tm_q / tm_do are make_row_map over q and dout as
+// T*H_q rows, tm_k / tm_v make_kv_map over k and v.
+cudaError_t launch_bwd_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                          const CUtensorMap& tm_do, const float2* stat, const SeqPlan& p, const int32_t* ptr,
                           const int32_t* rows, int h_q, int h_kv, int d, int block_size, float* dqacc, bf16* dk,
                           bf16* dv, int32_t* status, cudaStream_t st);
 

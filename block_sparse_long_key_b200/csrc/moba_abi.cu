@@ -53,7 +53,7 @@ struct PlanBufs {
 
 PlanBufs carve_plan(Carve& c, const moba_shape* s) {
   PlanBufs p;
-  p.status = c.take<int32_t>(1);
+  p.status = c.take<int32_t>(2);  // [0] status bits, [1] kernel-path bits
   p.cu = c.take<int32_t>(s->batch + 1);
   p.blk_off = c.take<int32_t>(s->batch + 1);
   p.tile_off = c.take<int32_t>(s->batch + 1);
@@ -107,7 +107,6 @@ struct BwdBufs {
   int32_t* cursor;
   int32_t* rows;
   int32_t* chunk_cnt;
-  float* dsum;
   float2* stat;  // (LSE, D) per row for the tcgen05 backward
   float* dqacc;
   float* dw_part;  // per-block key-conv dW partials (width <= 8)
@@ -124,7 +123,6 @@ BwdBufs carve_bwd(Carve& c, const moba_shape* s) {
   b.rows = c.take<int32_t>(nrow * s->topk);
   const size_t nch = moba::index_chunk_ints(s->total_tokens, s->h_kv, nb_max_of(s));
   b.chunk_cnt = nch ? c.take<int32_t>(nch) : nullptr;
-  b.dsum = c.take<float>(nrow);
   b.stat = c.take<float2>(nrow);
   b.dqacc = c.take<float>(nrow * s->head_dim);
   b.dw_part = c.take<float>((size_t)s->h_kv * nb_max_of(s) * s->head_dim * 8);
@@ -153,7 +151,7 @@ void stage_mark(int idx, cudaStream_t st) {
 int begin_plan(const PlanBufs& pb, const int32_t* cu_seqlens, const moba_shape* s, cudaStream_t st,
                moba::SeqPlan* plan, int stage) {
   STAGE_BEGIN(stage);
-  MOBA_TRY(cudaMemsetAsync(pb.status, 0, sizeof(int32_t), st));
+  MOBA_TRY(cudaMemsetAsync(pb.status, 0, 2 * sizeof(int32_t), st));
   MOBA_TRY(moba::launch_plan(cu_seqlens, s->batch, s->total_tokens, s->block_size, pb.cu, pb.blk_off, pb.tile_off,
                              pb.status, st));
   STAGE_END(stage);
@@ -261,19 +259,18 @@ int moba_forward(const void* q, const void* k, const void* v, const int32_t* cu_
                                     b.plan.status, st, b.chunk_cnt));
   STAGE_END(MOBA_STAGE_FWD_INDEX);
   STAGE_BEGIN(MOBA_STAGE_FWD_ATTN);
-  CUtensorMap tm_q;
-  if (moba::fwd_tc_supported(d, B) && moba::make_row_map(&tm_q, kq, (unsigned long long)T * hq, d) == cudaSuccess)
-    MOBA_TRY(moba::launch_fwd_tc(tm_q, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.lacc,
-                                 b.flag, b.plan.status, st));
-  else
-    MOBA_TRY(moba::launch_fwd_attn(kq, kk, kv, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.lacc, b.flag,
-                                   st));
+  CUtensorMap tm_q, tm_k, tm_v;
+  MOBA_TRY(moba::make_row_map(&tm_q, kq, (unsigned long long)T * hq, d));
+  MOBA_TRY(moba::make_kv_map(&tm_k, kk, T, hkv, d, B));
+  MOBA_TRY(moba::make_kv_map(&tm_v, kv, T, hkv, d, B));
+  MOBA_TRY(moba::launch_fwd_tc(tm_q, tm_k, tm_v, plan, b.ptr, b.rows, b.mref, hq, hkv, d, B, b.oacc, b.lacc, b.flag,
+                               b.plan.status, st));
   STAGE_END(MOBA_STAGE_FWD_ATTN);
   STAGE_BEGIN(MOBA_STAGE_FWD_FINALIZE);
   MOBA_TRY(moba::launch_fwd_finalize(b.oacc, b.lacc, b.mref, b.flag, T * hq, d, static_cast<bf16*>(out), lse,
                                      b.flag_list, st));
   MOBA_TRY(moba::launch_fwd_fallback(kq, kk, kv, plan, sel_idx, b.flag_list, hq, hkv, d, B, topk,
-                                     static_cast<bf16*>(out), lse, st));
+                                     static_cast<bf16*>(out), lse, b.plan.status, st));
   STAGE_END(MOBA_STAGE_FWD_FINALIZE);
   return MOBA_OK;
 }
@@ -329,22 +326,16 @@ int moba_backward(const void* q, const void* k, const void* v, const void* out, 
   STAGE_END(MOBA_STAGE_BWD_INDEX);
   STAGE_BEGIN(MOBA_STAGE_BWD_PRE);
   MOBA_TRY(moba::launch_bwd_pre(static_cast<const bf16*>(out), static_cast<const bf16*>(dout), lse, T * hq, d,
-                                b.dsum, b.stat, b.dqacc, st));
+                                b.stat, b.dqacc, st));
   STAGE_END(MOBA_STAGE_BWD_PRE);
   STAGE_BEGIN(MOBA_STAGE_BWD_ATTN);
-  CUtensorMap tm_q, tm_do;
-  if (moba::bwd_tc_supported(d, shape->block_size) &&
-      moba::make_row_map(&tm_q, q, (unsigned long long)T * hq, d) == cudaSuccess &&
-      moba::make_row_map(&tm_do, dout, (unsigned long long)T * hq, d) == cudaSuccess) {
-    MOBA_TRY(moba::launch_bwd_tc(tm_q, static_cast<const bf16*>(k), static_cast<const bf16*>(v), tm_do, b.stat,
-                                 plan, ptr, rows, hq, hkv, d, shape->block_size, b.dqacc, static_cast<bf16*>(dk),
-                                 static_cast<bf16*>(dv), b.plan.status, st));
-  } else {
-    MOBA_TRY(moba::launch_bwd_attn(static_cast<const bf16*>(q), static_cast<const bf16*>(k),
-                                   static_cast<const bf16*>(v), static_cast<const bf16*>(dout), lse, b.dsum, plan, ptr,
-                                   rows, hq, hkv, d, shape->block_size, b.dqacc, static_cast<bf16*>(dk),
-                                   static_cast<bf16*>(dv), st));
-  }
+  CUtensorMap tm_q, tm_do, tm_k, tm_v;
+  MOBA_TRY(moba::make_row_map(&tm_q, q, (unsigned long long)T * hq, d));
+  MOBA_TRY(moba::make_row_map(&tm_do, dout, (unsigned long long)T * hq, d));
+  MOBA_TRY(moba::make_kv_map(&tm_k, k, T, hkv, d, shape->block_size));
+  MOBA_TRY(moba::make_kv_map(&tm_v, v, T, hkv, d, shape->block_size));
+  MOBA_TRY(moba::launch_bwd_tc(tm_q, tm_k, tm_v, tm_do, b.stat, plan, ptr, rows, hq, hkv, d, shape->block_size,
+                               b.dqacc, static_cast<bf16*>(dk), static_cast<bf16*>(dv), b.plan.status, st));
   STAGE_END(MOBA_STAGE_BWD_ATTN);
   STAGE_BEGIN(MOBA_STAGE_BWD_DQ);
   MOBA_TRY(moba::launch_bwd_dq(b.dqacc, T * hq * d, static_cast<bf16*>(dq), st));
@@ -391,6 +382,18 @@ int moba_check_status(const void* workspace, void* stream, int32_t* device_statu
   if (cudaMemcpy(&v, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess) return MOBA_ELAUNCH;
   *device_status = v;
   return v ? MOBA_EDEVICE : MOBA_OK;
+}
+
+int moba_check_path(const void* workspace, void* stream, int32_t* path_bits) {
+  if (!workspace || !path_bits) return MOBA_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOBA_ELAUNCH;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, static_cast<const int32_t*>(workspace) + 1, sizeof(int32_t), cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return MOBA_ELAUNCH;
+  *path_bits = v;
+  return MOBA_OK;
 }
 
 const char* moba_status_string(int code) {

@@ -132,6 +132,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   uint64_t* bk = reinterpret_cast<uint64_t*>(sm + Ly::BK_OFF);
   const uint32_t mb_full = sbase + Ly::MB_OFF, mb_empty = mb_full + 8 * Ly::NB;
   const uint32_t mb_c0 = mb_empty + 8 * Ly::NB, mb_q = mb_c0 + 16;
+  mark_path(status, kPathRouteTc);
 
   const int ntiles = __ldg(tile_off + batch);
   // Longest rows first, every head's together: a CTA's time grows with its

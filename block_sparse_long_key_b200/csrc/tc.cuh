@@ -40,8 +40,16 @@ __device__ __forceinline__ uint32_t sw64_offset(int r, int c) {
   return (uint32_t)((r >> 3) * 512 + (r & 7) * 64 + ((c ^ ((r >> 1) & 3)) << 4));
 }
 
+// Byte offset of the 16-byte chunk `c` of row `r` in a SW32 region whose
+// rows are 32 bytes (16 bf16) wide: 8 rows per 256-byte atom, chunk c stored
+// at c ^ ((r / 4) % 2).
+__device__ __forceinline__ uint32_t sw32_offset(int r, int c) {
+  return (uint32_t)((r >> 3) * 256 + (r & 7) * 32 + ((c ^ ((r >> 2) & 1)) << 4));
+}
+
 constexpr uint32_t kLayoutSW128 = 2;
 constexpr uint32_t kLayoutSW64 = 4;
+constexpr uint32_t kLayoutSW32 = 6;
 
 // General shared-memory matrix descriptor.  K-major swizzled operands use
 // `sbo` = byte distance between 8-row groups (the leading offset is unused);
@@ -55,6 +63,48 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t smem_addr, uint32_t lbo, 
   d |= (uint64_t)1u << 46;
   d |= (uint64_t)layout << 61;
   return d;
+}
+
+// A tile of 128 rows x BLK keys (bf16; the P and dS tiles of the attention
+// kernels), keys contiguous in a row.  Rows up to 128 bytes wide use one
+// region with the widest swizzle that fits (32, 64 or 128 bytes); BLK = 128
+// uses two 128-byte-swizzled regions of 64 keys each, one after the other.
+template <int BLK>
+struct KeyTile {
+  static_assert(BLK == 16 || BLK == 32 || BLK == 64 || BLK == 128, "block size");
+  static constexpr uint32_t ROWB = BLK * 2 < 128 ? BLK * 2 : 128;  // bytes per row and region
+  static constexpr int NREG = BLK * 2 / (int)ROWB;
+  static constexpr uint32_t ATOM = 8 * ROWB;                       // one 8-row group
+  static constexpr uint32_t REGION = 128 * ROWB;
+  static constexpr uint32_t BYTES = NREG * REGION;
+  static constexpr uint32_t LAYOUT = BLK == 16 ? kLayoutSW32 : (BLK == 32 ? kLayoutSW64 : kLayoutSW128);
+  // Byte offset of the 16-byte chunk c (keys 8c .. 8c+7) of row r.
+  static __device__ __forceinline__ uint32_t offset(int r, int c) {
+    constexpr int CPR = (int)ROWB / 16;  // chunks per region row
+    const uint32_t reg = (uint32_t)(c / CPR) * REGION;
+    const int cc = c % CPR;
+    if constexpr (BLK == 16) return reg + sw32_offset(r, cc);
+    else if constexpr (BLK == 32) return reg + sw64_offset(r, cc);
+    else return reg + sw128_offset(r, cc);
+  }
+};
+
+// Zeroes rows [n, BLK) of a key block's K_j and V_j tiles (BLK rows, SW128
+// K-major, 64-wide d chunks as regions of BLK * 128 bytes): a partial last
+// block, where the TMA brought the next sequence's tokens or its zero fill,
+// so no value outside the block reaches an MMA.  Generic-proxy stores: the
+// caller fences them (fence_proxy_async) before the tensor cores read.
+template <int D, int BLK>
+__device__ __forceinline__ void zero_kv_tail_rows(unsigned char* k_tile, unsigned char* v_tile, int n, int tid,
+                                                  int nthreads) {
+  constexpr int KB = D / 64;
+  constexpr uint32_t KV_REGION = BLK * 128;
+  for (int i = tid; i < (BLK - n) * KB * 8; i += nthreads) {
+    const int r = n + i / (KB * 8), c = i % (KB * 8);
+    const uint32_t o = (c >> 3) * KV_REGION + sw128_offset(r, c & 7);
+    *reinterpret_cast<uint4*>(k_tile + o) = make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(v_tile + o) = make_uint4(0, 0, 0, 0);
+  }
 }
 
 // Instruction descriptor with the operand majorness: a_mn / b_mn = 1 when A
@@ -126,6 +176,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// 32 lanes x 16 consecutive columns (fp32).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+
 // 32 lanes x 32 consecutive columns: thread t writes its lane's columns.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
   asm volatile(
@@ -192,6 +252,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int 
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(mbar)
+      : "memory");
+}
+
+// TMA 3-D tile load: the box at (x, y, z) of `tmap` into shared memory at
+// `dst`, completion counted in bytes on `mbar`.  No cluster multicast.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int x, int y, int z, uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(mbar)
       : "memory");
 }
 

@@ -19,7 +19,8 @@ LIB_PATH = os.path.join(_PKG, "libmoba.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "moba.h")
 
 MOBA_OK, MOBA_EINVAL, MOBA_EALIGN, MOBA_EWORKSPACE, MOBA_ELAUNCH, MOBA_EDEVICE = 0, -1, -2, -3, -4, -5
-STATUS_BAD_SEQLENS, STATUS_BAD_SEL_IDX, STATUS_INDEX_OVERFLOW = 1, 2, 4
+STATUS_BAD_SEQLENS, STATUS_BAD_SEL_IDX, STATUS_INDEX_OVERFLOW, STATUS_TIMEOUT = 1, 2, 4, 8
+PATH_ROUTE_TCGEN05, PATH_FWD_TCGEN05, PATH_BWD_TCGEN05, PATH_EXACT_ROWS = 1, 2, 4, 8
 
 
 class Shape(ctypes.Structure):
@@ -70,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.moba_set_stage_events.restype = I
         L.moba_check_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
         L.moba_check_status.restype = I
+        L.moba_check_path.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
+        L.moba_check_path.restype = I
         L.moba_status_string.argtypes = [I]
         L.moba_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -271,4 +274,12 @@ def check_status(workspace: torch.Tensor) -> int:
     rc = lib().moba_check_status(_ptr(workspace), _stream(), ctypes.byref(st))
     if rc not in (MOBA_OK, MOBA_EDEVICE):
         raise MobaError(rc, "moba_check_status")
+    return int(st.value)
+
+
+def check_path(workspace: torch.Tensor) -> int:
+    """Synchronises the current stream and returns the kernel-path bits
+    (PATH_*) the last call on ``workspace`` set."""
+    st = ctypes.c_int32(0)
+    _check(lib().moba_check_path(_ptr(workspace), _stream(), ctypes.byref(st)), "moba_check_path")
     return int(st.value)

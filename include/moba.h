@@ -77,6 +77,13 @@ typedef struct moba_shape {
 #define MOBA_STATUS_INDEX_OVERFLOW 4
 #define MOBA_STATUS_TIMEOUT 8     /* a bounded device wait gave up; outputs of that call are invalid */
 
+/* Kernel-path bits reported by moba_check_path(): which kernel families the
+ * last call on a workspace ran (each kernel's first thread sets its bit). */
+#define MOBA_PATH_ROUTE_TCGEN05 1 /* routing scores on the tcgen05 tensor cores */
+#define MOBA_PATH_FWD_TCGEN05 2   /* forward attention on the tcgen05 tensor cores */
+#define MOBA_PATH_BWD_TCGEN05 4   /* backward attention on the tcgen05 tensor cores */
+#define MOBA_PATH_EXACT_ROWS 8    /* rows far above the softmax reference recomputed exactly */
+
 /* Bytes of device workspace moba_forward / moba_key_conv_centroid need for
  * `shape` (0 for an invalid shape).  The caller allocates it; its contents
  * need no initialisation and are scratch after the call, except the status
@@ -160,15 +167,20 @@ int moba_build_index(const int32_t* sel_idx, const int32_t* cu_seqlens, const mo
  * forbids side allocations, or latency-critical paths that must not call
  * cudaMalloc because it can synchronise the device.
  *
- * Same inputs, outputs and results as moba_build_index, without the
- * workspace: its scratch lives in a static device array of
- * MOBA_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that
- * loads the library keeps until the process exits.  The call allocates and
- * frees nothing.
+ * Same inputs and outputs as moba_build_index, without the workspace: its
+ * scratch lives in a static device array of MOBA_NOALLOC_SCRATCH_BYTES
+ * compiled into the library, which every GPU that loads the library keeps
+ * until the process exits.  The call allocates and frees nothing.  blk_ptr
+ * is identical to moba_build_index's and every bucket holds the same row
+ * ids, but the order of the ids inside a bucket may differ between the two
+ * entry points and from call to call (consumers only sum over a bucket).
  *
- *  - Runs on the current device; `stream` must belong to it.  The first call
- *    on each device looks up the array's device address (cudaGetSymbolAddress)
- *    and caches it; make that first call before any stream capture.
+ *  - Runs on the current device; `stream` must belong to it.  Every call
+ *    looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress, a host-side query), so a device reset never
+ *    leaves a stale address behind.  The first call on a device also makes
+ *    the runtime set the array up in that device's context: make it before
+ *    any stream capture.
  *  - Every call on a device shares the one array, and the array keeps what the
  *    last call left in it (this call clears what must start at zero).  Calls
  *    whose work overlaps on the GPU (other streams, other host threads) race
@@ -260,6 +272,14 @@ int moba_key_conv_backward(const void* k, const float* conv_w, int conv_width, c
  * Returns MOBA_OK, MOBA_EDEVICE if any bit is set, or MOBA_ELAUNCH if the
  * stream reported a CUDA error. */
 int moba_check_status(const void* workspace, void* stream, int32_t* device_status);
+
+/* Synchronises `stream`, then reads which kernel families the last call on
+ * this workspace ran (MOBA_PATH_* bits; forward workspace: routing, forward
+ * attention, exact rows; backward workspace: backward attention).  Returns
+ * MOBA_OK or MOBA_ELAUNCH if the stream reported a CUDA error.  Every shape
+ * the library accepts runs the tcgen05 kernels: there is no other attention
+ * or routing path. */
+int moba_check_path(const void* workspace, void* stream, int32_t* path_bits);
 
 /* Static description of a return code. */
 const char* moba_status_string(int code);

@@ -54,6 +54,7 @@ __all__ = [
     "silu",
     "key_conv",
     "block_centroids",
+    "past_block_scores",
     "route_row",
     "route",
     "visible_tokens",
@@ -149,6 +150,13 @@ def block_centroids(k: np.ndarray, cu_seqlens, block_size: int) -> List[np.ndarr
     return out
 
 
+def past_block_scores(q_i: np.ndarray, cent_h: np.ndarray, pos: int, block_size: int) -> np.ndarray:
+    """Router scores s_j = q_i . c_j of the earlier blocks j < pos // B of the
+    query at local position ``pos`` (§"Architettura del Modello Statistico"
+    1), in block order."""
+    return cent_h[: pos // block_size] @ q_i
+
+
 def route_row(q_i: np.ndarray, cent_h: np.ndarray, pos: int, block_size: int,
               topk: int) -> Tuple[List[int], float]:
     """Block selection of one query.
@@ -165,7 +173,7 @@ def route_row(q_i: np.ndarray, cent_h: np.ndarray, pos: int, block_size: int,
     b = pos // block_size
     if b == 0:
         return [0], math.inf
-    scores = cent_h[:b] @ q_i
+    scores = past_block_scores(q_i, cent_h, pos, block_size)
     order = sorted(range(b), key=lambda j: (-scores[j], j))
     keep = order[: topk - 1]
     gap = math.inf

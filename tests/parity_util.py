@@ -8,7 +8,8 @@ Tolerances (bf16 inputs, fp32 accumulation on the GPU, fp64 oracle):
 * O: max-abs <= 2e-2 and mean-abs <= 1e-3; LSE: max-abs <= 1e-3.
 * dQ/dK/dV, element by element: |g_gpu - g_ref| <= 4 u (s + |g_ref|) with
   u = 2^-8 (bf16 unit roundoff) and s the first-order rounding magnitude of
-  that element (``grad_error_scales``), plus mean-abs <= 4e-3 * rms(g_ref).
+  that element (``grad_error_scales``), plus mean-abs <= 2.5e-3 * rms(g_ref)
+  (measured on the B200 over every case: 1.1e-3 .. 1.9e-3).
   Derivation: the GPU rounds one factor of every product to bf16 before the
   MMAs (P for dV, dS for dQ and dK; fp32 sums), forms D_i = dO_i . O_i from
   the bf16 output O as the FlashAttention-style backward does, and rounds the
@@ -18,7 +19,13 @@ Tolerances (bf16 inputs, fp32 accumulation on the GPU, fp64 oracle):
   zero, so dQ can be far smaller than its terms); dK likewise with q, and
   dV by u * sum_i P_it |dO_ic|; each plus u |g| for the final rounding.  A
   numpy emulation of exactly those roundings reproduces the GPU values and
-  stays within 0.45 of this bound (of 4u) on the small cases.
+  stays within 0.45 of this bound (of 4u) on the small cases; the GPU itself
+  stays within 0.23 of it on every case, full-size key blocks included.
+  The mean-abs limit is above the 1e-3 * rms first proposed for the
+  gradients: rounding P and dS to bf16 (relative error up to u / 2 = 2^-9 per
+  factor) before the tensor-core products leaves a mean error of ~1.5e-3 of
+  the rms on these N(0, 1) inputs, the same as the FlashAttention-style
+  backward, whose bf16 P / dS it follows.
 """
 from __future__ import annotations
 
@@ -26,27 +33,83 @@ import numpy as np
 import torch
 
 from oracle import moba_oracle as orc
+from oracle import moba_oracle_c as orc_c
 
 GAP = 1e-3
 O_MAX, O_MEAN, LSE_MAX = 2e-2, 1e-3, 1e-3
 U_BF16 = 2.0 ** -8
-G_FACTOR, G_MEAN = 4.0, 4e-3
+G_FACTOR, G_MEAN = 4.0, 2.5e-3
 
 
 def to64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").double().numpy()
 
 
-def selection_mismatch_rows(sel_gpu: np.ndarray, sel_ref: np.ndarray, gap: np.ndarray, rows=None):
-    """Rows (t, h) whose GPU selection differs; asserts each is a near tie."""
+def check_near_tie_row(gpu_row, ref_row, scores, b: int, topk: int, what=""):
+    """A GPU selection that differs from the oracle's on a near-tie row must
+    still be a valid top-k selection that differs only inside the band.
+
+    ``scores``: the oracle's scores of the earlier blocks 0..b-1.  Checked:
+    exactly min(topk-1, b) earlier blocks plus the own block b, ascending
+    without repeats, b last, -1 padding after; every block the GPU kept and
+    the oracle did not (and every one the oracle kept and the GPU did not)
+    has a score within GAP (relative) of the oracle's threshold, the score of
+    its last kept earlier block.
+    """
+    gpu_row = [int(x) for x in gpu_row]
+    k1 = min(topk - 1, b)
+    valid = [x for x in gpu_row if x >= 0]
+    tag = (what, "gpu", gpu_row, "oracle", [int(x) for x in ref_row])
+    assert len(valid) == k1 + 1, ("wrong number of selected blocks",) + tag
+    assert gpu_row[len(valid):] == [-1] * (topk - len(valid)), ("padding",) + tag
+    assert valid == sorted(set(valid)), ("not ascending / repeated",) + tag
+    assert valid[-1] == b and all(0 <= j < b for j in valid[:-1]), ("own block / range",) + tag
+    ref_past = {int(x) for x in ref_row if 0 <= x < b}
+    gpu_past = set(valid[:-1])
+    thr = min(scores[j] for j in ref_past)
+    for j in (gpu_past - ref_past) | (ref_past - gpu_past):
+        assert abs(scores[j] - thr) <= GAP * max(abs(scores[j]), abs(thr)), \
+            ("swapped block outside the near-tie band", j, scores[j], thr) + tag
+
+
+def validate_selection_rows(sel_gpu_rows, sel_ref_rows, gap_rows, rows, q, cents, cu, block_size: int, topk: int,
+                            what=""):
+    """Compares GPU and oracle selections of the listed (token, head) rows
+    (row-aligned arrays [R, topk], gap [R]).
+
+    Rows must match exactly, except near ties (oracle gap <= GAP), whose GPU
+    selection must pass ``check_near_tie_row``.  Those excused rows are
+    returned, reported, and may be at most max(2, 1 %) of the rows compared.
+    ``q`` [T, H_q, d], ``cents`` the oracle's per-sequence centroid arrays.
+    """
+    cu = np.asarray(cu)
+    starts = cu[:-1]
+    g = q.shape[1] // cents[0].shape[0]
     bad = []
-    it = rows if rows is not None else [(t, h) for t in range(sel_ref.shape[0]) for h in range(sel_ref.shape[1])]
-    for t, h in it:
-        if not np.array_equal(sel_gpu[t, h], sel_ref[t, h]):
-            assert gap[t, h] <= GAP, ("selection differs outside the near-tie band", t, h, sel_gpu[t, h],
-                                      sel_ref[t, h], gap[t, h])
-            bad.append((t, h))
+    differ = np.nonzero((np.asarray(sel_gpu_rows) != np.asarray(sel_ref_rows)).any(axis=-1))[0]
+    for r in differ:
+        t, h = rows[r]
+        assert gap_rows[r] <= GAP, ("selection differs outside the near-tie band", what, t, h, sel_gpu_rows[r],
+                                    sel_ref_rows[r], gap_rows[r])
+        s = int(np.searchsorted(starts, t, side="right") - 1)
+        pos = t - int(cu[s])
+        scores = orc.past_block_scores(np.asarray(q[t, h], dtype=np.float64), cents[s][h // g], pos, block_size)
+        check_near_tie_row(sel_gpu_rows[r], sel_ref_rows[r], scores, pos // block_size, topk,
+                           "%s row %s" % (what, (t, h)))
+        bad.append((int(t), int(h)))
+    print("%s: %d of %d rows selected differently (near ties, validated)" % (what, len(bad), len(rows)))
+    assert len(bad) <= max(2, len(rows) // 100), (what, "too many near-tie rows", len(bad), len(rows))
     return bad
+
+
+def validate_selection(sel_gpu: np.ndarray, ref: dict, block_size: int, topk: int, rows=None, what=""):
+    """``validate_selection_rows`` over every row (or the listed rows) of
+    full [T, H_q, topk] arrays; ``ref`` is the dict of ``oracle_forward``."""
+    if rows is None:
+        rows = [(t, h) for t in range(ref["sel"].shape[0]) for h in range(ref["sel"].shape[1])]
+    idx = tuple(np.array(rows).T)
+    return validate_selection_rows(sel_gpu[idx], ref["sel"][idx], ref["gap"][idx], rows, ref["q"], ref["cents"],
+                                   ref["cu"], block_size, topk, what)
 
 
 def check_o_lse(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
@@ -66,6 +129,7 @@ def check_grad(g_gpu, g_ref, scale, what=""):
     assert np.isfinite(g_gpu).all(), what
     bound = G_FACTOR * U_BF16 * (scale + np.abs(g_ref)) + 1e-6 * rms
     ratio = err / bound
+    print("%s: max err/bound %.3f, mean-abs/rms %.2e" % (what, ratio.max(), err.mean() / rms))
     assert ratio.max() <= 1.0, (what, "max err / bound", ratio.max(), "max-abs/rms", err.max() / rms)
     assert err.mean() <= G_MEAN * rms, (what, "mean-abs/rms", err.mean() / rms)
     return ratio.max(), err.mean() / rms
@@ -119,15 +183,16 @@ def row_dq_error_scale(q, k, v, dout, sel, cu, B, rows, o_rows, lse_rows):
     return out
 
 
-def oracle_forward(x: dict, B: int, topk: int, rows=None):
-    """Oracle k', centroids, selection (+gap), O, LSE from CPU inputs."""
+def oracle_forward(x: dict, B: int, topk: int, rows=None, impl=orc_c):
+    """Oracle k', centroids, selection (+gap), O, LSE from CPU inputs (the
+    fp64 C++ oracle by default; ``impl=orc`` for the numpy one)."""
     cu = x["cu_seqlens"].numpy()
     q = x["q"].double().numpy()
     k = x["k"].double().numpy()
     v = x["v"].double().numpy()
     if "conv_w" in x:
-        k = orc.key_conv(k, x["conv_w"].double().numpy(), cu)
-    cents = orc.block_centroids(k, cu, B)
-    sel, gap = orc.route(q, cents, cu, B, topk, rows=rows)
-    o, lse = orc.attention(q, k, v, sel, cu, B, rows=rows)
+        k = impl.key_conv(k, x["conv_w"].double().numpy(), cu)
+    cents = impl.block_centroids(k, cu, B)
+    sel, gap = impl.route(q, cents, cu, B, topk, rows=rows)
+    o, lse = impl.attention(q, k, v, sel, cu, B, rows=rows)
     return dict(k=k, cents=cents, sel=sel, gap=gap, o=o, lse=lse, q=q, v=v, cu=cu)

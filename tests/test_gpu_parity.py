@@ -1,13 +1,17 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
 the same seeded inputs.  Small cases compare every element; the full-size
-workloads compare seeded samples of rows the oracle computes one by one."""
+workloads compare seeded samples of rows, and dK / dV of chosen key blocks,
+that the oracle computes one by one.  Every case also checks which kernel
+families ran (the tcgen05 router and attention kernels)."""
 import numpy as np
 import pytest
 import torch
 
 from block_sparse_long_key_b200 import moba, synth
-from oracle import moba_oracle as orc
+from oracle import moba_oracle_c as orc
 import parity_util as pu
+
+FWD_PATH = moba.PATH_ROUTE_TCGEN05 | moba.PATH_FWD_TCGEN05
 
 pytestmark = pytest.mark.gpu
 
@@ -45,16 +49,24 @@ def _gpu(x, dev):
     return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
 
 
+def _forward(g, w, workspace=None):
+    shape = moba.shape_of(g["q"], g["k"], g["cu_seqlens"], w.block_size, w.topk)
+    ws = workspace if workspace is not None else moba.alloc_workspace(moba.fwd_workspace_size(shape), g["q"].device)
+    res = moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], w.block_size, w.topk, conv_w=g.get("conv_w"),
+                       workspace=ws)
+    return res, ws
+
+
 @pytest.mark.parametrize("case", SMALL, ids=_ids)
 def test_forward_matches_oracle(dev, case):
     w, x = _inputs(case)
     g = _gpu(x, dev)
-    out, lse, sel, _ = moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], w.block_size, w.topk,
-                                    conv_w=g.get("conv_w"))
-    torch.cuda.synchronize()
+    (out, lse, sel, _), ws = _forward(g, w)
+    assert moba.check_status(ws) == 0
+    assert moba.check_path(ws) & FWD_PATH == FWD_PATH, moba.check_path(ws)
     ref = pu.oracle_forward(x, w.block_size, w.topk)
     sel_g = sel.cpu().numpy()
-    bad = pu.selection_mismatch_rows(sel_g, ref["sel"], ref["gap"])
+    bad = pu.validate_selection(sel_g, ref, w.block_size, w.topk, what=_ids(case))
     o_g, lse_g = pu.to64(out), pu.to64(lse)
     o_ref, lse_ref = ref["o"].copy(), ref["lse"].copy()
     if bad:   # near ties: re-check those rows under the GPU's own selection
@@ -160,12 +172,15 @@ def test_block_index_large_block_counts(dev, seqlen):
 def test_backward_matches_oracle(dev, case):
     w, x = _inputs(case)
     g = _gpu(x, dev)
-    out, lse, sel, k_used = moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], w.block_size, w.topk,
-                                         conv_w=g.get("conv_w"))
-    dq, dk, dv = moba.backward(g["q"], k_used, g["v"], out, lse, g["dout"], sel, g["cu_seqlens"], w.block_size)
-    torch.cuda.synchronize()
+    (out, lse, sel, k_used), _ = _forward(g, w)
+    shape = moba.shape_of(g["q"], g["k"], g["cu_seqlens"], w.block_size, w.topk)
+    ws_b = moba.alloc_workspace(moba.bwd_workspace_size(shape), dev)
+    dq, dk, dv = moba.backward(g["q"], k_used, g["v"], out, lse, g["dout"], sel, g["cu_seqlens"], w.block_size,
+                               workspace=ws_b)
+    assert moba.check_status(ws_b) == 0
+    assert moba.check_path(ws_b) & moba.PATH_BWD_TCGEN05, moba.check_path(ws_b)
     ref = pu.oracle_forward(x, w.block_size, w.topk)
-    bad = pu.selection_mismatch_rows(sel.cpu().numpy(), ref["sel"], ref["gap"])
+    bad = pu.validate_selection(sel.cpu().numpy(), ref, w.block_size, w.topk, what=_ids(case))
     do64 = x["dout"].double().numpy()
     dq_r, dk_r, dv_r = orc.attention_backward(ref["q"], ref["k"], ref["v"], do64, ref["sel"], ref["cu"], w.block_size)
     sq, sk, sv = pu.grad_error_scales(ref["q"], ref["k"], ref["v"], do64, ref["sel"], ref["cu"], w.block_size,
@@ -235,42 +250,95 @@ def _sample_rows(w, per_head, seed):
     rows = []
     for h in range(w.h_q):
         ts = r.choice(w.total_tokens, size=min(per_head, w.total_tokens), replace=False)
-        rows += [(int(t), h) for t in ts]
+        rows += [(int(t), h) for t in sorted(ts)]
     return rows
+
+
+def _check_blocks(w, seed):
+    """Key blocks whose dK / dV are compared at full size, per checked KV head:
+    the first four of each sequence (the longest buckets, the longest CTAs),
+    the last one inside the window the attention kernels issue early, one in
+    the middle, the last two (the last may be partial) and two at random."""
+    r = np.random.default_rng(seed)
+    nbs = [(L + w.block_size - 1) // w.block_size for L in w.seqlens]
+    nb_max = w.total_tokens // w.block_size + w.batch
+    offs = np.concatenate([[0], np.cumsum(nbs)])
+    kvs = sorted({0, w.h_kv - 1}) if w.h_q == w.h_kv else [w.h_kv - 1]
+    blocks = []
+    for kv in kvs:
+        for s, n in enumerate(nbs):
+            js = {0, 1, 3, max(nb_max // 8 - 1, 0), n // 2, n - 2, n - 1, int(r.integers(0, max(n, 1)))}
+            blocks += [(kv, int(offs[s] + j)) for j in sorted(js) if 0 <= j < n]
+    return blocks, offs
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("name", list(synth.WORKLOADS))
 def test_full_size_sampled_rows(dev, name):
     w = synth.WORKLOADS[name]
+    B, topk = w.block_size, w.topk
     x = synth.make_inputs(w)
     g = _gpu(x, dev)
-    out, lse, sel, k_used = moba.forward(g["q"], g["k"], g["v"], g["cu_seqlens"], w.block_size, w.topk,
-                                         conv_w=g.get("conv_w"))
+    (out, lse, sel, k_used), ws = _forward(g, w)
+    assert moba.check_status(ws) == 0
+    assert moba.check_path(ws) & FWD_PATH == FWD_PATH
     dq = None
     if w.backward:
-        dq, dk, dv = moba.backward(g["q"], k_used, g["v"], out, lse, g["dout"], sel, g["cu_seqlens"], w.block_size)
-        assert torch.isfinite(dk.float()).all() and torch.isfinite(dv.float()).all()
+        shape = moba.shape_of(g["q"], g["k"], g["cu_seqlens"], B, topk)
+        ws_b = moba.alloc_workspace(moba.bwd_workspace_size(shape), dev)
+        dq, dk, dv = moba.backward(g["q"], k_used, g["v"], out, lse, g["dout"], sel, g["cu_seqlens"], B,
+                                   workspace=ws_b)
+        assert moba.check_status(ws_b) == 0
+        assert moba.check_path(ws_b) & moba.PATH_BWD_TCGEN05
     torch.cuda.synchronize()
-    rows = _sample_rows(w, 48, 7)
-    ref = pu.oracle_forward(x, w.block_size, w.topk, rows=rows)
-    sel_g = sel.cpu().numpy()
-    bad = pu.selection_mismatch_rows(sel_g, ref["sel"], ref["gap"], rows=rows)
-    o_g, lse_g = pu.to64(out), pu.to64(lse)
-    sel_use = ref["sel"].copy()
-    for t, h in bad:
-        sel_use[t, h] = sel_g[t, h]
-    o_ref, lse_ref = orc.attention(ref["q"], ref["k"], ref["v"], sel_use, ref["cu"], w.block_size, rows=rows)
+    del g
+    cu = x["cu_seqlens"].numpy()
+    q = x["q"].double().numpy()
+    k = x["k"].double().numpy()
+    if "conv_w" in x:
+        k = orc.key_conv(k, x["conv_w"].double().numpy(), cu)
+    v = x["v"].double().numpy()
+    cents = orc.block_centroids(k, cu, B)
+    rows = _sample_rows(w, 512, 7)
     idx = tuple(np.array(rows).T)
-    pu.check_o_lse(o_g[idx], lse_g[idx], o_ref[idx], lse_ref[idx], name)
+    sel_all = sel.cpu().numpy()
+    sel_g = sel_all[idx]
+    sel_r, gap_r = orc.route_rows(q, cents, cu, B, topk, rows)
+    bad = pu.validate_selection_rows(sel_g, sel_r, gap_r, rows, q, cents, cu, B, topk, what=name)
+    sel_use = sel_r.copy()
+    for i, (t, h) in enumerate(rows):           # near ties: re-checked under the GPU's selection
+        if (t, h) in bad:
+            sel_use[i] = sel_g[i]
+    o_ref, lse_ref = orc.attention_rows(q, k, v, sel_use, cu, B, rows)
+    pu.check_o_lse(pu.to64(out)[idx], pu.to64(lse)[idx], o_ref, lse_ref, name)
     for kv, hq, i, j in x["needles"]:          # planted blocks are always picked
-        assert j in sel_g[i, hq], (kv, hq, i, j)
-    if dq is not None:
-        do32 = x["dout"].float().numpy()
-        dq_r, _ = orc.backward_rows(ref["q"], ref["k"], ref["v"], do32, sel_use, ref["cu"], w.block_size, rows)
-        s_r = pu.row_dq_error_scale(ref["q"], ref["k"], ref["v"], do32, sel_use, ref["cu"], w.block_size, rows,
-                                    o_ref[idx], lse_ref[idx])
-        pu.check_grad(pu.to64(dq)[idx], dq_r, s_r, "dq " + name)
+        assert j in sel_all[i, hq], (kv, hq, i, j)
+    if w.total_tokens * w.h_q <= (1 << 21):     # every row's selection where the oracle is quick enough
+        every = [(t, h) for t in range(w.total_tokens) for h in range(w.h_q)]
+        sel_full, gap_full = orc.route(q, cents, cu, B, topk)
+        pu.validate_selection_rows(sel_all.reshape(-1, topk), sel_full.reshape(-1, topk), gap_full.reshape(-1),
+                                   every, q, cents, cu, B, topk, what=name + " all rows")
+    if dq is None:
+        return
+    do = x["dout"].double().numpy()
+    dq_r = orc.backward_rows(q, k, v, do, sel_use, cu, B, rows)
+    s_r = pu.row_dq_error_scale(q, k, v, do, sel_all, cu, B, rows, o_ref, lse_ref)
+    pu.check_grad(pu.to64(dq)[idx], dq_r, s_r, "dq " + name)
+    # dK / dV of chosen key blocks, under the GPU's own selection of every
+    # query (its agreement with the oracle's is checked on the rows above).
+    blocks, offs = _check_blocks(w, 11)
+    dk_r, dv_r, sk, sv = orc.block_grads(q, k, v, do, sel_all, cu, B, blocks, magnitudes=True)
+    dk_g, dv_g = pu.to64(dk), pu.to64(dv)
+    gk, gv, rk, rv, ak, av = [], [], [], [], [], []
+    for i, (kv, gb) in enumerate(blocks):
+        s = int(np.searchsorted(offs, gb, side="right") - 1)
+        t0 = int(cu[s]) + (gb - int(offs[s])) * B
+        t1 = min(t0 + B, int(cu[s + 1]))
+        gk.append(dk_g[t0:t1, kv]); gv.append(dv_g[t0:t1, kv])
+        rk.append(dk_r[i, :t1 - t0]); rv.append(dv_r[i, :t1 - t0])
+        ak.append(sk[i, :t1 - t0]); av.append(sv[i, :t1 - t0])
+    pu.check_grad(np.concatenate(gk), np.concatenate(rk), np.concatenate(ak), "dk blocks " + name)
+    pu.check_grad(np.concatenate(gv), np.concatenate(rv), np.concatenate(av), "dv blocks " + name)
 
 
 @pytest.mark.parametrize("case", [SMALL[1], SMALL[3]], ids=_ids)
@@ -285,7 +353,7 @@ def test_backward_reusing_forward_index_matches_oracle(dev, case):
                                fwd_workspace=wsf)
     torch.cuda.synchronize()
     ref = pu.oracle_forward(x, w.block_size, w.topk)
-    assert not pu.selection_mismatch_rows(sel.cpu().numpy(), ref["sel"], ref["gap"])
+    assert not pu.validate_selection(sel.cpu().numpy(), ref, w.block_size, w.topk, what="reuse")
     do64 = x["dout"].double().numpy()
     dq_r, dk_r, dv_r = orc.attention_backward(ref["q"], ref["k"], ref["v"], do64, ref["sel"], ref["cu"], w.block_size)
     sq, sk, sv = pu.grad_error_scales(ref["q"], ref["k"], ref["v"], do64, ref["sel"], ref["cu"], w.block_size,
@@ -329,7 +397,7 @@ def test_rows_far_above_the_reference_take_the_exact_path(dev, d, B):
     ref = pu.oracle_forward(x, B, w.topk)
     assert j in ref["sel"][i, h]               # the planted block is picked by that query
     sel_g = sel.cpu().numpy()
-    bad = pu.selection_mismatch_rows(sel_g, ref["sel"], ref["gap"])   # near ties only
+    bad = pu.validate_selection(sel_g, ref, B, w.topk, what="overflow")   # near ties only
     o_g, lse_g = pu.to64(out), pu.to64(lse)
     assert np.isfinite(o_g).all() and np.isfinite(lse_g).all()
     assert lse_g[i, h] > 100.0                 # the huge logit dominates

@@ -2,9 +2,10 @@
 library device scratch memory (a host framework that owns every byte of
 device memory, or a latency-critical path that must not call cudaMalloc).
 
-It must return exactly what the workspace version, moba_build_index,
-returns, call after call, although every call reuses the same static scratch
-array.  This file is collected last on purpose; it also passes when run on
+It must return what the workspace version, moba_build_index, returns (the
+same bucket offsets and, per bucket, the same row ids; their order inside a
+bucket is unspecified), call after call, although every call reuses the same
+static scratch array.  This file is collected last on purpose; it also passes when run on
 its own in a fresh process.
 """
 import ctypes
