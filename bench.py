@@ -15,7 +15,8 @@ fraction of the measured B200 bf16 tensor peak.
 With N > 1 (launched by torchrun) every rank runs its own independent
 problem of the same shape (different seeds): no data-path collective; the
 step time is the max over ranks and ``value`` the aggregate throughput.
-``--impl reference`` times the fp64 CPU oracle on a bounded sample instead.
+``--impl reference`` times the fp64 C++ CPU oracle (every host core) on a
+bounded sample instead.
 """
 from __future__ import annotations
 
@@ -48,11 +49,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel source file it was taken with: a changed source voids the figure.
 # Headline workload, one timed-step launch each (profiles/dram_traffic_n64k_h16_d64_b32_k32_kconv4.md).
 NCU_TRAFFIC = {
-    "fwd_route": {"bytes": 278.41e6 + 366.40e6, "sha": "41a06d3978d3dcd1"},
-    "fwd_attn": {"bytes": 1.1695e9 + 722.40e6, "sha": "4c84aea0e6808372"},
-    "bwd_attn": {"bytes": 1.9538e9 + 1.0273e9, "sha": "fb01b862248ff62e"},
-    "conv_bwd": {"bytes": 268.46e6 + 126.76e6, "sha": "2e8a64640582a328"},
-    "fwd_centroid": {"bytes": 134.25e6 + 102.10e6, "sha": "103ae9898d36c11f"},
+    "fwd_route": {"bytes": 278.22e6 + 366.72e6, "sha": "6cb84cd7d1226227"},
+    "fwd_attn": {"bytes": 1.1706e9 + 719.20e6, "sha": "5b561e1c286c88a7"},
+    "bwd_attn": {"bytes": 1.9063e9 + 1.0038e9, "sha": "3ffdaa36749d5531"},
+    "conv_bwd": {"bytes": 268.46e6 + 127.35e6, "sha": "2e8a64640582a328"},
+    "fwd_centroid": {"bytes": 134.26e6 + 101.85e6, "sha": "103ae9898d36c11f"},
 }
 
 
@@ -170,7 +171,7 @@ def stage_roofline(name, w, pairs, scored, peaks):
     if name == "fwd_finalize":
         return "hbm", T * hq * (d * 6.0 + 12), "byte"
     if name == "bwd_pre":
-        return "hbm", T * hq * (d * 8.0 + 4), "byte"
+        return "hbm", T * hq * (d * 8.0 + 12), "byte"
     if name == "bwd_dq":
         return "hbm", T * hq * d * 6.0, "byte"
     if name in ("fwd_index", "bwd_index"):
@@ -194,12 +195,24 @@ LAUNCHES_CONV_BWD = 3
 
 # ----------------------------------------------------------------------------- oracle (CPU) timing
 
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def oracle_sample(w: synth.Workload, seed: int, rows_per_step: int, steps: int, warmup: int):
-    """Times the fp64 oracle on sampled query rows.  Returns per-step TFLOP/s
-    values and a description.  Routing, attention and the per-row backward
-    run inside the timed region; the key conv and centroids (O(N d), computed
-    once for the whole input) are prepared outside it."""
-    from oracle import moba_oracle as orc
+    """Times the fp64 C++ oracle (OpenMP over rows, every host core) on
+    seeded samples of (query, head) rows.  Returns per-step TFLOP/s values,
+    a description and the thread count.  Routing against all past centroids,
+    attention and the per-row backward run inside the timed region; the key
+    conv and centroids (O(N d), computed once for the whole input) are
+    prepared outside it."""
+    from oracle import moba_oracle_c as orc
 
     x = synth.make_inputs(w, seed=seed)
     cu = x["cu_seqlens"].numpy()
@@ -211,32 +224,25 @@ def oracle_sample(w: synth.Workload, seed: int, rows_per_step: int, steps: int, 
     dout = x["dout"].double().numpy()
     cents = orc.block_centroids(k, cu, w.block_size)
     r = np.random.default_rng(seed)
+    n = min(rows_per_step, w.total_tokens * w.h_q)
+    flops_row = 3.5 * 4.0 * w.topk * w.block_size * w.head_dim
     vals = []
-    cpu0, wall0 = time.process_time(), time.perf_counter()
     for step in range(warmup + steps):
-        ts = r.integers(0, w.total_tokens, rows_per_step)
-        hs = r.integers(0, w.h_q, rows_per_step)
-        rows = list(zip(ts.tolist(), hs.tolist()))
+        flat = r.choice(w.total_tokens * w.h_q, size=n, replace=False)
+        rows = [(int(f) // w.h_q, int(f) % w.h_q) for f in np.sort(flat)]
         t0 = time.perf_counter()
-        sel = np.full((w.total_tokens, w.h_q, w.topk), -1, dtype=np.int64)
-        starts = cu[:-1]
-        g = w.h_q // w.h_kv
-        useful = 0.0
-        for t, h in rows:
-            s = int(np.searchsorted(starts, t, side="right") - 1)
-            blocks, _ = orc.route_row(q[t, h], cents[s][h // g], t - int(cu[s]), w.block_size, w.topk)
-            sel[t, h, :len(blocks)] = blocks
-            useful += 3.5 * 4.0 * w.topk * w.block_size * w.head_dim
-        orc.attention(q, k, v, sel, cu, w.block_size, rows=rows)
+        sel, _ = orc.route_rows(q, cents, cu, w.block_size, w.topk, rows)
+        orc.attention_rows(q, k, v, sel, cu, w.block_size, rows)
         orc.backward_rows(q, k, v, dout, sel, cu, w.block_size, rows)
         dt = time.perf_counter() - t0
         if step >= warmup:
-            vals.append(useful / dt / 1e12)
-    cores = max(1, round((time.process_time() - cpu0) / max(time.perf_counter() - wall0, 1e-9)))
-    desc = ("%d random (query, head) rows per step: routing against all past centroids, attention and the "
-            "per-row backward in fp64 numpy; FLOPs counted as 3.5*4*k*B*d per row (nominal, as on the GPU); "
-            "key conv and centroids prepared outside the timed region" % rows_per_step)
-    return vals, desc, cores
+            vals.append(n * flops_row / dt / 1e12)
+    threads = orc.num_threads()
+    desc = ("%d random (query, head) rows per step (of %d) through the fp64 C++ oracle, OpenMP on %d threads "
+            "(host: %d cores, %s): routing against all past centroids, attention and the per-row backward; "
+            "FLOPs counted as 3.5*4*k*B*d per row (nominal, as on the GPU); key conv and centroids prepared "
+            "outside the timed region" % (n, w.total_tokens * w.h_q, threads, os.cpu_count() or 0, cpu_model()))
+    return vals, desc, threads
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -471,9 +477,9 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        vals, desc, cores = oracle_sample(w, seed, args.cpu_rows, 2, 1)
+        vals, desc, cores = oracle_sample(w, seed, args.cpu_rows, 1, 0)
         cpu = {"value": round(statistics.mean(vals), 9), "unit": UNIT, "cores": cores, "kind": "oracle",
-               "sample": desc}
+               "sample": desc, "nproc": os.cpu_count(), "cpu_model": cpu_model()}
 
     if world > 1:
         dist.barrier()
@@ -519,7 +525,8 @@ def run_reference(args):
                        "h_kv": w.h_kv, "head_dim": w.head_dim, "block_size": w.block_size, "topk": w.topk,
                        "conv_width": w.conv_width, "needles_per_head": w.needles_per_head,
                        "sample_rows_per_step": args.ref_rows},
-            "cpu_baseline": {"value": round(v, 9), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": round(v, 9), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+                             "nproc": os.cpu_count(), "cpu_model": cpu_model()},
             "e2e": {"value": round(v, 9), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -536,8 +543,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention context timing")
-    ap.add_argument("--cpu-rows", type=int, default=1500, help="oracle rows per CPU-baseline step")
-    ap.add_argument("--ref-rows", type=int, default=400, help="oracle rows per --impl reference step")
+    ap.add_argument("--cpu-rows", type=int, default=65536, help="oracle rows per CPU-baseline step")
+    ap.add_argument("--ref-rows", type=int, default=4096, help="oracle rows per --impl reference step")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")

@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.moba_set_stage_events.restype = I
         L.moba_check_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
         L.moba_check_status.restype = I
+        L.moba_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, P, S, P]
+        L.moba_selftest_bounded_wait.restype = I
         L.moba_check_path.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
         L.moba_check_path.restype = I
         L.moba_status_string.argtypes = [I]
@@ -283,3 +285,10 @@ def check_path(workspace: torch.Tensor) -> int:
     st = ctypes.c_int32(0)
     _check(lib().moba_check_path(_ptr(workspace), _stream(), ctypes.byref(st)), "moba_check_path")
     return int(st.value)
+
+
+def selftest_bounded_wait(limit_ns: int, workspace: torch.Tensor) -> None:
+    """Runs the bounded-wait self-test kernel (see moba_selftest_bounded_wait)
+    on the current stream; read the outcome with ``check_status``."""
+    _check(lib().moba_selftest_bounded_wait(int(limit_ns), _ptr(workspace), workspace.numel(), _stream()),
+           "moba_selftest_bounded_wait")

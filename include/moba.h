@@ -281,6 +281,20 @@ int moba_check_status(const void* workspace, void* stream, int32_t* device_statu
  * or routing path. */
 int moba_check_path(const void* workspace, void* stream, int32_t* path_bits);
 
+/*
+ * Self-test of the bounded device waits (the pages have no counterpart).
+ * Every tensor-core kernel of this library waits on mbarriers for TMA copies,
+ * MMA completions and hand-offs between warps; each such wait gives up after
+ * a wall-clock limit, records MOBA_STATUS_TIMEOUT and lets the kernel return,
+ * so a lost completion cannot hang the GPU.  This entry point runs that path
+ * on purpose: one CTA waits, with limit `limit_ns` (1 ns .. 10 s), on an
+ * mbarrier that is never completed (no copy or MMA is in flight), then sets
+ * MOBA_STATUS_TIMEOUT in the status word of `workspace` (>= 256 bytes,
+ * 256-byte aligned; only its first 8 bytes are written) and exits.  Read the
+ * result with moba_check_status(); the device stays usable afterwards.
+ */
+int moba_selftest_bounded_wait(unsigned long long limit_ns, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Static description of a return code. */
 const char* moba_status_string(int code);
 

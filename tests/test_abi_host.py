@@ -85,6 +85,12 @@ def test_argument_errors_return_codes_without_a_device(L):
     assert L.moba_key_conv_centroid(ok, None, 0, ok, ctypes.byref(s), None, None, ok, big, None) == moba.MOBA_EINVAL
     st = ctypes.c_int32(0)
     assert L.moba_check_status(None, None, ctypes.byref(st)) == moba.MOBA_EINVAL
+    assert L.moba_check_path(None, None, ctypes.byref(st)) == moba.MOBA_EINVAL
+    sw = L.moba_selftest_bounded_wait
+    assert sw(0, ok, 256, None) == moba.MOBA_EINVAL                 # a limit of 0 ns
+    assert sw(1 << 40, ok, 256, None) == moba.MOBA_EINVAL           # beyond 10 s
+    assert sw(1000, ok, 16, None) == moba.MOBA_EINVAL               # workspace too small
+    assert sw(1000, mis, 256, None) == moba.MOBA_EALIGN
 
 
 def test_binding_refuses_cpu_tensors():

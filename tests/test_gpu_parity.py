@@ -454,3 +454,24 @@ def test_forward_backward_replay_from_a_cuda_graph(dev):
         # fp32 reductions may add in another order: compare to bf16 resolution
         assert (a.float() - b.float()).abs().max().item() <= 2e-2 * max(1.0, b.float().abs().max().item())
     del graph
+
+
+def test_bounded_wait_gives_up_and_reports_a_timeout(dev):
+    # A device wait that can never complete (an mbarrier short of one
+    # arrival, nothing in flight) must give up after its limit, record
+    # MOBA_STATUS_TIMEOUT and return; the next call on a fresh workspace
+    # runs clean.
+    ws = moba.alloc_workspace(256, dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    moba.selftest_bounded_wait(1_000_000, ws)          # 1 ms
+    e1.record()
+    assert moba.check_status(ws) == moba.STATUS_TIMEOUT
+    ms = e0.elapsed_time(e1)
+    assert 1.0 <= ms < 500.0, ms
+    w, x = _inputs(((512,), 2, 2, 64, 32, 4, 0))
+    g = _gpu(x, dev)
+    (out, lse, sel, _), ws2 = _forward(g, w)
+    assert moba.check_status(ws2) == 0
+    assert moba.check_path(ws2) & FWD_PATH == FWD_PATH
+    assert torch.isfinite(out.float()).all()
