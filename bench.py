@@ -12,9 +12,11 @@ fraction of the measured B200 bf16 tensor peak.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-With N > 1 (launched by torchrun) every rank runs its own independent
-problem of the same shape (different seeds): no data-path collective; the
-step time is the max over ranks and ``value`` the aggregate throughput.
+With N > 1 (launched by torchrun) the KV-head groups of one seeded problem
+are split over the ranks (a KV head and its query heads stay together, so no
+data-path collective is needed; strong scaling); ``--shard replica`` runs an
+independent problem of the same shape per rank instead (weak scaling).  The
+step time is the max over ranks and ``value`` the whole job's throughput.
 ``--impl reference`` times the fp64 C++ CPU oracle (every host core) on a
 bounded sample instead.
 """
@@ -148,13 +150,39 @@ def reduce_max(value: float, device, world: int) -> float:
     return float(t.item())
 
 
-def aggregate_value(flops_per_step_per_rank: float, world: int, ms_per_step: float) -> float:
+def aggregate_value(total_flops_per_step: float, ms_per_step: float) -> float:
     """Whole-job TFLOP/s: every rank's work over the slowest rank's time."""
-    return flops_per_step_per_rank * world / (ms_per_step * 1e-3) / 1e12
+    return total_flops_per_step / (ms_per_step * 1e-3) / 1e12
 
 
 def rank_seed(w: synth.Workload, rank: int) -> int:
     return w.seed + 7919 * rank
+
+
+def head_shard(h_kv: int, world: int, rank: int):
+    """KV heads [kv0, kv1) of rank `rank` when one problem's KV-head groups
+    are split over `world` ranks: contiguous ranges, the first h_kv % world
+    ranks taking one more.  A KV head and the query heads that read it stay
+    on one rank, so dK / dV never cross ranks and the path needs no
+    collective."""
+    base, extra = divmod(h_kv, world)
+    kv0 = rank * base + min(rank, extra)
+    return kv0, kv0 + base + (1 if rank < extra else 0)
+
+
+def shard_inputs(x: dict, w: synth.Workload, kv0: int, kv1: int):
+    """The inputs of KV heads [kv0, kv1) (and their query heads) of one
+    problem, as contiguous tensors, and the workload they form."""
+    import dataclasses
+    g = w.h_q // w.h_kv
+    out = {"q": x["q"][:, kv0 * g:kv1 * g].contiguous(), "k": x["k"][:, kv0:kv1].contiguous(),
+           "v": x["v"][:, kv0:kv1].contiguous(), "cu_seqlens": x["cu_seqlens"],
+           "needles": [(kv - kv0, hq - kv0 * g, i, j) for kv, hq, i, j in x["needles"] if kv0 <= kv < kv1]}
+    if "dout" in x:
+        out["dout"] = x["dout"][:, kv0 * g:kv1 * g].contiguous()
+    if "conv_w" in x:
+        out["conv_w"] = x["conv_w"][kv0:kv1].contiguous()
+    return out, dataclasses.replace(w, h_kv=kv1 - kv0, h_q=(kv1 - kv0) * g)
 
 
 def stage_roofline(name, w, pairs, scored, peaks):
@@ -293,8 +321,19 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     moba.lib()
 
-    seed = rank_seed(w, rank)
-    x = synth.make_inputs(w, seed=seed)
+    # N > 1: KV-head groups of one problem split over the ranks (strong
+    # scaling, the default), or one independent problem per rank.
+    sharded = world > 1 and args.shard == "heads" and w.h_kv >= world
+    total_flops = (w.fwd_flops() + w.bwd_flops()) * (1 if sharded else world)
+    if sharded:
+        seed = w.seed
+        kv0, kv1 = head_shard(w.h_kv, world, rank)
+        x, w = shard_inputs(synth.make_inputs(w, seed=seed), w, kv0, kv1)
+        parallelism = "KV-head groups of one problem sharded over %d GPUs, no collective" % world
+    else:
+        seed = rank_seed(w, rank)
+        x = synth.make_inputs(w, seed=seed)
+        parallelism = "independent problem per GPU" if world > 1 else "single GPU"
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     T, hq, hkv, d, B, topk = w.total_tokens, w.h_q, w.h_kv, w.head_dim, w.block_size, w.topk
     shape = moba.shape_of(g["q"], g["k"], g["cu_seqlens"], B, topk)
@@ -351,8 +390,7 @@ def run_ours(args):
     fwd_ms = sum(v for k_, v in stage_ms.items() if k_.startswith("fwd"))
     bwd_ms = sum(v for k_, v in stage_ms.items() if k_.startswith("bwd") or k_ == "conv_bwd")
 
-    flops = w.fwd_flops() + w.bwd_flops()
-    value = aggregate_value(flops, world, ms_max)
+    value = aggregate_value(total_flops, ms_max)
     peak_t = float(peaks["bf16_tflops"])
 
     dom = max(stage_ms, key=stage_ms.get)
@@ -463,7 +501,7 @@ def run_ours(args):
         e1.record(s_out)
         torch.cuda.synchronize()
         ems = reduce_max(e0.elapsed_time(e1) / ne, dev, world)
-        e2e = {"value": round(aggregate_value(flops, world, ems), 3), "unit": UNIT, "ms_per_step": round(ems, 3),
+        e2e = {"value": round(aggregate_value(total_flops, ems), 3), "unit": UNIT, "ms_per_step": round(ems, 3),
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": ne,
                "pipelining": "inputs/outputs double-buffered; upload, kernels, download on three streams"}
         if moba.check_status(ws_f) | moba.check_status(ws_b):
@@ -487,13 +525,14 @@ def run_ours(args):
         in_bytes = sum(g[n].numel() * g[n].element_size() for n in ("q", "k", "v", "dout"))
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True,
+            "scaling": "strong" if sharded else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "seq_len": T, "batch": w.batch, "h_q": hq, "h_kv": hkv, "head_dim": d,
                        "block_size": B, "topk": topk, "conv_width": w.conv_width,
                        "needles_per_head": w.needles_per_head,
                        "l2": "inputs %.0f MB > %d MB L2 (no flush)" % (in_bytes / 1e6, L2_BYTES >> 20),
-                       "parallelism": "independent problem per GPU" if world > 1 else "single GPU"},
+                       "parallelism": parallelism},
             "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
             "fwd_tflops": round(w.fwd_flops() / (fwd_ms * 1e-3) / 1e12, 3),
             "bwd_tflops": round(w.bwd_flops() / (bwd_ms * 1e-3) / 1e12, 3),
@@ -538,6 +577,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(synth.WORKLOADS), default=synth.HEADLINE)
+    ap.add_argument("--shard", choices=["heads", "replica"], default="heads",
+                    help="N > 1: split one problem's KV-head groups over the ranks, or run one problem per rank")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the KV head count (query heads scale with it); for small profiling runs")
     ap.add_argument("--no-e2e", action="store_true")
