@@ -34,6 +34,14 @@
 // end each thread sorts its row's kept block indices in registers and writes
 // the row.
 //
+// Tiles whose rows scan at least kTwoPassMinChunks chunks run two passes over
+// the chunks.  The first keeps, per row, the ceil((k-1)/2) largest of its
+// chunks' second-largest scores; the smallest of those is a lower bound lb of
+// the row's (k-1)-th best score (at least k-1 scores reach it).  The second
+// pass replays the same MMAs (bit-identical scores) and sends to the heap
+// only scores >= lb, so the selection stays exact while the heap admits ~50
+// instead of ~140 scores per row of 1024 candidates.
+//
 // Side outputs for the forward: mref = a lower bound of the query's largest
 // attention logit, max(best kept score, q_i.k_i) / sqrt(d) (a block mean never
 // exceeds the block max), the fixed softmax reference of the forward; the
@@ -54,6 +62,10 @@ constexpr uint64_t kKeyMax = ~0ull;  // heap padding: never the minimum
 constexpr uint64_t kKeyEmpty = (uint64_t)0x007fffffu << 32;
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr int kGroup = 4;  // columns appended between buffer checks
+constexpr int kBoundList = 16;  // chunk second-maxima kept for the bound: ceil((k-1)/2) <= 16
+// Tiles whose rows scan fewer chunks route in one pass: the bound needs at
+// least ceil((k-1)/2) chunks and saves little on short rows.
+constexpr int kTwoPassMinChunks = 16;
 
 template <int D, int NC, int LISTN>
 struct RouteLayout {
@@ -65,7 +77,7 @@ struct RouteLayout {
   static constexpr uint32_t C_MAT = KB * C_REGION;       // hi or lo of one chunk
   static constexpr uint32_t C_BUF = 2 * C_MAT;           // hi + lo
   static constexpr uint32_t HP_OFF = C_OFF + 2 * C_BUF;           // heap keys [LISTN][kSel] u64
-  static constexpr uint32_t BK_OFF = HP_OFF + LISTN * kSel * 8;  // candidate keys [kBuf][kSel] u64
+  static constexpr uint32_t BK_OFF = HP_OFF + LISTN * kSel * 8;  // candidates [kBuf][kSel] (score bits, index)
   // mbarriers: score tile full [NB] (MMA done), score tile empty [NB] (read
   // by the four selecting warps), chunk landed [2], Q in tensor memory.
   static constexpr uint32_t MB_OFF = BK_OFF + kBuf * kSel * 8;
@@ -129,7 +141,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   unsigned char* sm = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
   const uint32_t sbase = smem_u32(sm);
   uint64_t* heap = reinterpret_cast<uint64_t*>(sm + Ly::HP_OFF);
-  uint64_t* bk = reinterpret_cast<uint64_t*>(sm + Ly::BK_OFF);
+  uint2* bk = reinterpret_cast<uint2*>(sm + Ly::BK_OFF);
   const uint32_t mb_full = sbase + Ly::MB_OFF, mb_empty = mb_full + 8 * Ly::NB;
   const uint32_t mb_c0 = mb_empty + 8 * Ly::NB, mb_q = mb_c0 + 16;
   mark_path(status, kPathRouteTc);
@@ -151,6 +163,14 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   const int k1 = topk - 1;
   const int nscan = k1 > 0 ? (p0 + nrows - 1) / block_size : 0;  // blocks any row may score
   const int nchunks = (nscan + NC - 1) / NC;
+  // Two passes over the chunks when the rows are long enough: the first only
+  // computes a lower bound of each row's (k-1)-th best score, the second
+  // replays the same MMAs (bit-identical scores) and admits into the heap
+  // only the scores at or above that bound.  See pass_one below.
+  const int k2 = (k1 + 1) / 2;
+  const bool two_pass = LISTN == 32 && k1 >= 2 && nchunks >= kTwoPassMinChunks;
+  const int nsteps = two_pass ? 2 * nchunks : nchunks;
+  auto chunk_of = [&](int st) { return st < nchunks ? st : st - nchunks; };
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t qstride = (size_t)h_q * D;
 
@@ -179,6 +199,11 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
     for (int sl = 0; sl < LISTN; ++sl) heap[sl * kSel + tid] = sl < k1 ? kKeyEmpty : kKeyMax;
   uint64_t root_key = kKeyEmpty;  // the heap's root: the worst kept key
   float tau = -INFINITY;          // its score
+  float lb = -INFINITY;           // the first pass's lower bound (two-pass tiles)
+  // Candidates pass when x > thr = max(tau, the float just below lb): x > tau
+  // (strict: blocks arrive in ascending j, so a score equal to the root's,
+  // which has a lower index, never wins) and x >= lb in one compare.
+  float thr = -INFINITY;
   int cnt = 0;                    // buffered candidate keys
   if (tid == 0) {
     for (int i = 0; i < Ly::NB; ++i) {
@@ -204,8 +229,8 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   __syncthreads();
   tc::fence_after_sync();
   const bool producer = tid == kSel;  // lane 0 of the last warp
-  if (producer && nchunks > 0) load_chunk(0, 0);
-  if (producer && nchunks > 1) load_chunk(1, 1);
+  if (producer && nsteps > 0) load_chunk(chunk_of(0), 0);
+  if (producer && nsteps > 1) load_chunk(chunk_of(1), 1);
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
   constexpr uint32_t idesc = tc::idesc_bf16_f32(kTM, NC);
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -283,37 +308,55 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
       heap[pos * kSel + tid] = key;
       root_key = root;
       tau = from_order_bits((uint32_t)(root >> 32));
+      thr = fmaxf(tau, nextafterf(lb, -INFINITY));
     }
   };
   // One round: every thread with buffered keys admits its latest one (full
   // keys are compared, so the order of admission does not matter).  Rounds
   // run only while some thread's buffer is close to full, so most threads
   // have work in each of them.
+  // Candidates wait in the buffer as (score bits, block index); the heap key
+  // is built only for the one a round admits.
   auto flush_round = [&]() {
     const bool has = cnt > 0;
     cnt -= has ? 1 : 0;
-    const uint64_t key = bk[cnt * kSel + tid];  // slot 0 when empty: read, not used
+    const uint2 e = bk[cnt * kSel + tid];  // slot 0 when empty: read, not used
+    const uint64_t key = make_key(__uint_as_float(e.x), (int)e.y);
     admit(key, has && key > root_key);
   };
 
-  // Selection on one chunk's scores: those above the row's threshold go to
-  // the candidate buffer, which the warp flushes into the heaps in rounds.
-  auto select_scores = [&](const uint32_t (&v)[NC], int c) {
+  // Lower bound of the row's (k-1)-th best score (first pass).  The row
+  // keeps the k2 = ceil((k-1)/2) largest of its chunks' second-largest
+  // scores; the k2-th of them, lb, is met or beaten by at least two scores in
+  // each of k2 chunks, so at least k-1 scores of the row are >= lb: every
+  // block of the row's top k-1 has a score >= lb, and a second pass that
+  // admits only scores >= lb still selects exactly (the second pass replays
+  // the same MMAs, so its scores are bit-identical).  On N(0, 1)-like scores
+  // about 50 of 1024 scores pass it, against ~140 heap admissions for a plain
+  // running threshold.
+
+  const int wmin_b = __shfl_sync(kFull, my_b, 0);  // smallest own block of the warp's rows (lane 0's)
+
+  // Selection on one chunk's scores: those above the row's threshold (and
+  // the first pass's bound) go to the candidate buffer, which the warp
+  // flushes into the heaps in rounds.
+  auto select_scores = [&](uint32_t (&v)[NC], int c) {
     const int jbase = c * NC;
+    if (jbase + NC > wmin_b) {  // blocks at or after a row's own block lie in this chunk
+      const int lim = my_b - jbase;
+#pragma unroll
+      for (int col = 0; col < NC; ++col) v[col] = col < lim ? v[col] : 0xff800000u;  // -inf
+    }
 #pragma unroll
     for (int g = 0; g < NC / kGroup; ++g) {
       while (__any_sync(kFull, cnt > Ly::kBuf - kGroup)) flush_round();  // room for the next group
 #pragma unroll
       for (int e = 0; e < kGroup; ++e) {
         const int col = g * kGroup + e;
-        const float x = __uint_as_float(v[col]);
-        const int j = jbase + col;
-        // Blocks arrive in ascending j, so a score equal to tau (the root's,
-        // which has a lower index) never wins: the strict test is exact.
-        // Branch-free: slot cnt is free (cnt < kBuf here), so the key is
-        // stored either way and only counted when it passes.
-        bk[cnt * kSel + tid] = make_key(x, j);
-        cnt += (j < my_b && x > tau) ? 1 : 0;
+        // Branch-free: slot cnt is free (cnt < kBuf here), so the candidate
+        // is stored either way and only counted when it passes.
+        bk[cnt * kSel + tid] = make_uint2(v[col], (uint32_t)(jbase + col));
+        cnt += __uint_as_float(v[col]) > thr ? 1 : 0;
       }
     }
   };
@@ -327,14 +370,15 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   // chunks.  Every wait is bounded and decided warp-wide; one that gives up
   // ends the loop, and the block agrees on the outcome afterwards.
   bool ok = true;
-  if (producer && nchunks > 0) {
+  if (producer && nsteps > 0) {
     ok = tc::mbar_wait(mb_q, 0);
-    for (int c = 0; c < nchunks && ok; ++c) {
+    // step c of the (one or two) passes: chunk chunk_of(c)
+    for (int c = 0; c < nsteps && ok; ++c) {
       const int buf = c & 1, sc = c % Ly::NB;
-      if (c >= 1 && c + 1 < nchunks) {
+      if (c >= 1 && c + 1 < nsteps) {
         const int pc = c - 1;
         if (!(ok = tc::mbar_wait(mb_full + 8 * (pc % Ly::NB), (pc / Ly::NB) & 1))) break;
-        load_chunk(c + 1, (c + 1) & 1);
+        load_chunk(chunk_of(c + 1), (c + 1) & 1);
       }
       if (!(ok = tc::mbar_wait(mb_c0 + 8 * buf, (c >> 1) & 1))) break;
       if (c >= Ly::NB && !(ok = tc::mbar_wait(mb_empty + 8 * sc, ((c / Ly::NB) - 1) & 1))) break;
@@ -356,15 +400,12 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
       tc::mma_commit(mb_full + 8 * sc);
     }
   } else if (sel_thread) {
-    for (int c = 0; c < nchunks; ++c) {
+    // Waits for score tile c % NB, reads it into registers and releases it.
+    auto take_tile = [&](int c, uint32_t (&v)[NC]) -> bool {
       const int sc = c % Ly::NB;
       const bool got = tc::mbar_wait(mb_full + 8 * sc, (c / Ly::NB) & 1);
-      if (!__all_sync(kFull, got)) {
-        ok = false;
-        break;
-      }
+      if (!__all_sync(kFull, got)) return false;
       tc::fence_after_sync();
-      uint32_t v[NC];
       const uint32_t taddr = tmem + lane_base + (uint32_t)(sc * NC);
 #pragma unroll
       for (int hf = 0; hf < NC / 32; ++hf)
@@ -373,7 +414,64 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(mb_empty + 8 * sc);
-      select_scores(v, c);
+      return true;
+    };
+    int c = 0;
+    if (two_pass) {
+      // First pass: the bound.  Every chunk of NC blocks contributes its
+      // second-largest score m2 (masked to the row's earlier blocks); the row
+      // keeps the kBoundList largest m2 in a descending register list.
+      float top2[kBoundList];
+#pragma unroll
+      for (int i = 0; i < kBoundList; ++i) top2[i] = -INFINITY;
+      for (; c < nchunks; ++c) {
+        uint32_t v[NC];
+        if (!take_tile(c, v)) {
+          ok = false;
+          break;
+        }
+        const int jbase = c * NC;
+        if (jbase + NC > wmin_b) {  // blocks at or after the row's own block count as -inf
+          const int lim = my_b - jbase;
+#pragma unroll
+          for (int col = 0; col < NC; ++col) v[col] = col < lim ? v[col] : 0xff800000u;
+        }
+        // second-largest of the chunk: pairwise (hi, lo), then merged top-2 lists
+        float hi[NC / 2], lo[NC / 2];
+#pragma unroll
+        for (int i = 0; i < NC / 2; ++i) {
+          const float a = __uint_as_float(v[2 * i]), b = __uint_as_float(v[2 * i + 1]);
+          hi[i] = fmaxf(a, b);
+          lo[i] = fminf(a, b);
+        }
+#pragma unroll
+        for (int w = NC / 4; w >= 1; w >>= 1)
+#pragma unroll
+          for (int i = 0; i < w; ++i) {
+            const float h2 = fmaxf(hi[i], hi[i + w]);
+            lo[i] = fmaxf(fminf(hi[i], hi[i + w]), fmaxf(lo[i], lo[i + w]));
+            hi[i] = h2;
+          }
+        const float m2 = lo[0];
+        // insert m2 into the descending list, dropping its smallest entry
+#pragma unroll
+        for (int i = kBoundList - 1; i >= 1; --i) top2[i] = fmaxf(top2[i], fminf(top2[i - 1], m2));
+        top2[0] = fmaxf(top2[0], m2);
+      }
+      // the k2-th largest: the list is descending, so the least of its first k2
+      lb = INFINITY;
+#pragma unroll
+      for (int i = 0; i < kBoundList; ++i) lb = i < k2 ? fminf(lb, top2[i]) : lb;
+      thr = fmaxf(tau, nextafterf(lb, -INFINITY));
+    }
+    // (Second) pass: selection into the heap.
+    for (; ok && c < nsteps; ++c) {
+      uint32_t v[NC];
+      if (!take_tile(c, v)) {
+        ok = false;
+        break;
+      }
+      select_scores(v, chunk_of(c));
     }
     if (ok)
       while (__any_sync(kFull, cnt > 0)) flush_round();
