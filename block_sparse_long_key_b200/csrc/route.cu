@@ -34,7 +34,7 @@
 // end each thread sorts its row's kept block indices in registers and writes
 // the row.
 //
-// Tiles whose rows scan at least kTwoPassMinChunks chunks run two passes over
+// At d = 64, tiles whose rows scan at least kTwoPassMinChunks chunks run two passes over
 // the chunks.  The first keeps, per row, the ceil((k-1)/2) largest of its
 // chunks' second-largest scores; the smallest of those is a lower bound lb of
 // the row's (k-1)-th best score (at least k-1 scores reach it).  The second
@@ -64,7 +64,10 @@ constexpr uint32_t kFull = 0xffffffffu;
 constexpr int kGroup = 4;  // columns appended between buffer checks
 constexpr int kBoundList = 16;  // chunk second-maxima kept for the bound: ceil((k-1)/2) <= 16
 // Tiles whose rows scan fewer chunks route in one pass: the bound needs at
-// least ceil((k-1)/2) chunks and saves little on short rows.
+// least ceil((k-1)/2) chunks and saves little on short rows.  At d = 128 the
+// replayed MMAs (twice the K steps) cost more than the admissions saved
+// (N = 256K, k = 16: 4.76 ms in one pass against 6.44 ms in two), so only
+// d = 64 tiles take two passes.
 constexpr int kTwoPassMinChunks = 16;
 
 template <int D, int NC, int LISTN>
@@ -168,7 +171,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   // replays the same MMAs (bit-identical scores) and admits into the heap
   // only the scores at or above that bound.  See pass_one below.
   const int k2 = (k1 + 1) / 2;
-  const bool two_pass = LISTN == 32 && k1 >= 2 && nchunks >= kTwoPassMinChunks;
+  const bool two_pass = D == 64 && LISTN == 32 && k1 >= 2 && nchunks >= kTwoPassMinChunks;
   const int nsteps = two_pass ? 2 * nchunks : nchunks;
   auto chunk_of = [&](int st) { return st < nchunks ? st : st - nchunks; };
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
