@@ -401,7 +401,8 @@ def run_ours(args):
     else:
         achieved = amount / (stage_ms[dom] * 1e-3) / 1e9
         peak, runit = float(peaks["hbm_gbs"]), "GB/s"
-    tr = NCU_TRAFFIC.get(dom)
+    # the captured traffic is for one launch of the headline workload on one GPU
+    tr = NCU_TRAFFIC.get(dom) if args.workload == synth.HEADLINE and not sharded else None
     traffic = tr["bytes"] if tr and tr.get("sha") == src_sha(KERNEL_SRC.get(dom, "fwd.cu")) else None
     roofline = {"kernel": dom, "bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": runit,
                 "frac": round(achieved / peak, 4), "traffic": traffic,
