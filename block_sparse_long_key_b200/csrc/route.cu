@@ -14,7 +14,7 @@
 //
 // One CTA owns 128 consecutive queries of one sequence and one query head.
 // Their Q tile sits in tensor memory (thread t writes row t, the MMA's A
-// operand); a stream of centroid chunks (NC blocks each, double buffered,
+// operand); a stream of centroid chunks (NC blocks each, kCB = 2 buffers,
 // TMA tile loads into 128-byte-swizzled K-major shared memory) is the B operand of
 // tcgen05.mma (M = 128 queries, N = NC blocks, bf16 in, fp32 accumulate into
 // tensor memory, three score tiles at d = 64, two at d = 128): a producer
@@ -79,12 +79,13 @@ struct RouteLayout {
   static constexpr uint32_t C_REGION = NC * 128;
   static constexpr uint32_t C_MAT = KB * C_REGION;       // hi or lo of one chunk
   static constexpr uint32_t C_BUF = 2 * C_MAT;           // hi + lo
-  static constexpr uint32_t HP_OFF = C_OFF + 2 * C_BUF;           // heap keys [LISTN][kSel] u64
+  static constexpr int kCB = 2;                           // chunk buffers (loads in flight)
+  static constexpr uint32_t HP_OFF = C_OFF + kCB * C_BUF;         // heap keys [LISTN][kSel] u64
   static constexpr uint32_t BK_OFF = HP_OFF + LISTN * kSel * 8;  // candidates [kBuf][kSel] (score bits, index)
   // mbarriers: score tile full [NB] (MMA done), score tile empty [NB] (read
   // by the four selecting warps), chunk landed [2], Q in tensor memory.
   static constexpr uint32_t MB_OFF = BK_OFF + kBuf * kSel * 8;
-  static constexpr uint32_t HOLD_OFF = MB_OFF + 8 * (2 * NB + 3);
+  static constexpr uint32_t HOLD_OFF = MB_OFF + 8 * (2 * NB + kCB + 1);
   static constexpr uint32_t BYTES = HOLD_OFF + 16;
   // Tensor memory: NB NC-column score tiles, then Q (D bf16 = D/2 columns).
   static constexpr uint32_t TM_Q = NB * NC;
@@ -146,7 +147,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   uint64_t* heap = reinterpret_cast<uint64_t*>(sm + Ly::HP_OFF);
   uint2* bk = reinterpret_cast<uint2*>(sm + Ly::BK_OFF);
   const uint32_t mb_full = sbase + Ly::MB_OFF, mb_empty = mb_full + 8 * Ly::NB;
-  const uint32_t mb_c0 = mb_empty + 8 * Ly::NB, mb_q = mb_c0 + 16;
+  const uint32_t mb_c0 = mb_empty + 8 * Ly::NB, mb_q = mb_c0 + 8 * Ly::kCB;
   mark_path(status, kPathRouteTc);
 
   const int ntiles = __ldg(tile_off + batch);
@@ -213,8 +214,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
       tc::mbar_init(mb_full + 8 * i, 1);
       tc::mbar_init(mb_empty + 8 * i, kSel / 32);
     }
-    tc::mbar_init(mb_c0, 1);
-    tc::mbar_init(mb_c0 + 8, 1);
+    for (int b = 0; b < Ly::kCB; ++b) tc::mbar_init(mb_c0 + 8 * b, 1);
     tc::mbar_init(mb_q, kSel / 32);
     tc::mbar_init_fence();
   }
@@ -232,8 +232,8 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   __syncthreads();
   tc::fence_after_sync();
   const bool producer = tid == kSel;  // lane 0 of the last warp
-  if (producer && nsteps > 0) load_chunk(chunk_of(0), 0);
-  if (producer && nsteps > 1) load_chunk(chunk_of(1), 1);
+  if (producer)
+    for (int b = 0; b < Ly::kCB && b < nsteps; ++b) load_chunk(chunk_of(b), b);
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
   constexpr uint32_t idesc = tc::idesc_bf16_f32(kTM, NC);
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -377,13 +377,14 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
     ok = tc::mbar_wait(mb_q, 0);
     // step c of the (one or two) passes: chunk chunk_of(c)
     for (int c = 0; c < nsteps && ok; ++c) {
-      const int buf = c & 1, sc = c % Ly::NB;
-      if (c >= 1 && c + 1 < nsteps) {
+      const int buf = c % Ly::kCB, sc = c % Ly::NB;
+      if (c >= 1 && c + Ly::kCB - 1 < nsteps) {
+        // chunk c - 1's MMAs are done with its buffer: load chunk c + kCB - 1 there
         const int pc = c - 1;
         if (!(ok = tc::mbar_wait(mb_full + 8 * (pc % Ly::NB), (pc / Ly::NB) & 1))) break;
-        load_chunk(chunk_of(c + 1), (c + 1) & 1);
+        load_chunk(chunk_of(c + Ly::kCB - 1), pc % Ly::kCB);
       }
-      if (!(ok = tc::mbar_wait(mb_c0 + 8 * buf, (c >> 1) & 1))) break;
+      if (!(ok = tc::mbar_wait(mb_c0 + 8 * buf, (c / Ly::kCB) & 1))) break;
       if (c >= Ly::NB && !(ok = tc::mbar_wait(mb_empty + 8 * sc, ((c / Ly::NB) - 1) & 1))) break;
       tc::fence_after_sync();
       const uint32_t d_tmem = tmem + (uint32_t)(sc * NC);
@@ -489,7 +490,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
     if (producer) {
       for (int i = 0; i < Ly::NB; ++i)
         for (int ph = 0; ph < 2; ++ph) tc::mbar_wait(mb_full + 8 * i, ph, 20000000ull);
-      for (int b2 = 0; b2 < 2; ++b2)
+      for (int b2 = 0; b2 < Ly::kCB; ++b2)
         for (int ph = 0; ph < 2; ++ph) tc::mbar_wait(mb_c0 + 8 * b2, ph, 20000000ull);
     }
     __syncthreads();
