@@ -193,7 +193,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (it + 1 < ntiles) gather(nrid);
     float l = 0.f, mx = -INFINITY;
     {
+      // keys of this block the row may see: all of a block in its past, the
+      // first (tok - t0 + 1) of its own block, none for a missing row
       const int tok = rid >= 0 ? rid / h_q : -1;
+      const int nvis = max(0, min(tok + 1, t1) - t0);
 #pragma unroll
       for (int h = 0; h < BLK / CW; ++h) {
         uint32_t sv[CW];
@@ -206,9 +209,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           float p2[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int key_tok = t0 + h * CW + c + u;
+            const int kk = h * CW + c + u;  // key index inside the block
             float p = 0.f;
-            if (key_tok <= tok && key_tok < t1) {
+            if (kk < nvis) {
               const float x = __uint_as_float(sv[c + u]) * scale_log2;
               p = fast_exp2(x - mr_c);
               mx = fmaxf(mx, x);
