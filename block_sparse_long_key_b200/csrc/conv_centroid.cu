@@ -42,7 +42,8 @@ template <int D, int W, int BLK>
 __global__ void __launch_bounds__(kThreads)
 conv_centroid_kernel(const bf16* __restrict__ k, const float* __restrict__ conv_w, const int32_t* __restrict__ cu,
                      const int32_t* __restrict__ blk_off, int batch, int nb_max, int h_kv, bf16* __restrict__ k_out,
-                     float* __restrict__ cent, bf16* __restrict__ cent_hi, bf16* __restrict__ cent_lo) {
+                     float* __restrict__ cent, bf16* __restrict__ cent_hi, bf16* __restrict__ cent_lo,
+                     float* __restrict__ cent_norm_max) {
   using Ly = CcLayout<D, W, BLK>;
   extern __shared__ __align__(16) unsigned char smem[];
   bf16* in = reinterpret_cast<bf16*>(smem);                    // [ROWS][SEG]
@@ -107,19 +108,34 @@ conv_centroid_kernel(const bf16* __restrict__ k, const float* __restrict__ conv_
             *reinterpret_cast<const uint4*>(outt + r * Ly::SEG + cc * 8);
     }
   }
+  const float cv = h < h_kv ? acc / (float)n : 0.f;
   if (h < h_kv) {
-    const float cv = acc / (float)n;
     const bf16 hb = __float2bfloat16_rn(cv);
     const size_t o = ((size_t)h * nb_max + gb) * D + c;
     cent[o] = cv;
     cent_hi[o] = hb;
     cent_lo[o] = __float2bfloat16_rn(cv - __bfloat162float(hb));
   }
+  if (cent_norm_max) {
+    // Largest centroid norm of each KV head (the router's screen pass bounds
+    // the part of a score it leaves out by it): a head's D channels are
+    // D / 32 whole warps; their squares meet in shared memory.
+    __shared__ float nrm2[Ly::HG];
+    if (tid < Ly::HG) nrm2[tid] = 0.f;
+    __syncthreads();
+    float sq = cv * cv;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    if ((tid & 31) == 0) atomicAdd(&nrm2[ch / D], sq);
+    __syncthreads();
+    if (tid < nh)  // non-negative floats order like their bit patterns
+      atomicMax(reinterpret_cast<int*>(cent_norm_max) + h0 + tid, __float_as_int(sqrtf(nrm2[tid])));
+  }
 }
 
 template <int D, int W>
 cudaError_t launch_cc_w(const bf16* k, const float* conv_w, const SeqPlan& p, int h_kv, int block_size, bf16* k_out,
-                        float* cent, bf16* cent_hi, bf16* cent_lo, cudaStream_t st) {
+                        float* cent, bf16* cent_hi, bf16* cent_lo, float* cnorm, cudaStream_t st) {
   const dim3 grid(p.nb_max, (h_kv + kThreads / D - 1) / (kThreads / D));
 #define MOBA_CC(BB)                                                                                      \
   {                                                                                                      \
@@ -128,7 +144,7 @@ cudaError_t launch_cc_w(const bf16* k, const float* conv_w, const SeqPlan& p, in
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
     if (e != cudaSuccess) return e;                                                                      \
     kern<<<grid, kThreads, smem, st>>>(k, conv_w, p.cu, p.blk_off, p.batch, p.nb_max, h_kv, k_out, cent,  \
-                                       cent_hi, cent_lo);                                                \
+                                       cent_hi, cent_lo, cnorm);                                         \
     return cudaGetLastError();                                                                           \
   }
   switch (block_size) {
@@ -143,17 +159,18 @@ cudaError_t launch_cc_w(const bf16* k, const float* conv_w, const SeqPlan& p, in
 
 template <int D>
 cudaError_t launch_cc_d(const bf16* k, const float* conv_w, int conv_width, const SeqPlan& p, int h_kv,
-                        int block_size, bf16* k_out, float* cent, bf16* cent_hi, bf16* cent_lo, cudaStream_t st) {
+                        int block_size, bf16* k_out, float* cent, bf16* cent_hi, bf16* cent_lo, float* cnorm,
+                        cudaStream_t st) {
   switch (conv_width) {
-    case 0: return launch_cc_w<D, 0>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
-    case 1: return launch_cc_w<D, 1>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
-    case 2: return launch_cc_w<D, 2>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
-    case 3: return launch_cc_w<D, 3>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
-    case 4: return launch_cc_w<D, 4>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
-    case 5: return launch_cc_w<D, 5>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
-    case 6: return launch_cc_w<D, 6>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
-    case 7: return launch_cc_w<D, 7>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
-    case 8: return launch_cc_w<D, 8>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
+    case 0: return launch_cc_w<D, 0>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, cnorm, st);
+    case 1: return launch_cc_w<D, 1>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, cnorm, st);
+    case 2: return launch_cc_w<D, 2>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, cnorm, st);
+    case 3: return launch_cc_w<D, 3>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, cnorm, st);
+    case 4: return launch_cc_w<D, 4>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, cnorm, st);
+    case 5: return launch_cc_w<D, 5>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, cnorm, st);
+    case 6: return launch_cc_w<D, 6>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, cnorm, st);
+    case 7: return launch_cc_w<D, 7>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, cnorm, st);
+    case 8: return launch_cc_w<D, 8>(k, conv_w, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, cnorm, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -162,11 +179,14 @@ cudaError_t launch_cc_d(const bf16* k, const float* conv_w, int conv_width, cons
 
 cudaError_t launch_conv_centroid(const bf16* k, const float* conv_w, int conv_width, const SeqPlan& p,
                                  int h_kv, int d, int block_size, bf16* k_out, float* cent,
-                                 bf16* cent_hi, bf16* cent_lo, cudaStream_t st) {
+                                 bf16* cent_hi, bf16* cent_lo, float* cent_norm_max, cudaStream_t st) {
   if (conv_width < 0 || conv_width > kMaxWidth || block_size > kMaxBlock) return cudaErrorInvalidValue;
   if (p.nb_max == 0 || h_kv == 0) return cudaSuccess;
-  if (d == 64) return launch_cc_d<64>(k, conv_w, conv_width, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
-  return launch_cc_d<128>(k, conv_w, conv_width, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, st);
+  if (d == 64)
+    return launch_cc_d<64>(k, conv_w, conv_width, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, cent_norm_max,
+                           st);
+  return launch_cc_d<128>(k, conv_w, conv_width, p, h_kv, block_size, k_out, cent, cent_hi, cent_lo, cent_norm_max,
+                          st);
 }
 
 }  // namespace moba

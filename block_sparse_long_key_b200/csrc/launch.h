@@ -29,9 +29,11 @@ cudaError_t launch_plan(const int32_t* cu_in, int batch, int total_tokens, int b
                         int32_t* cu_out, int32_t* blk_off, int32_t* tile_off, int32_t* status,
                         cudaStream_t st);
 
+// cent_norm_max (optional, h_kv floats, zeroed by the caller): receives each
+// KV head's largest centroid 2-norm.
 cudaError_t launch_conv_centroid(const bf16* k, const float* conv_w, int conv_width, const SeqPlan& p,
                                  int h_kv, int d, int block_size, bf16* k_out, float* cent,
-                                 bf16* cent_hi, bf16* cent_lo, cudaStream_t st);
+                                 bf16* cent_hi, bf16* cent_lo, float* cent_norm_max, cudaStream_t st);
 
 // Forward accumulator: rows of d floats (the unnormalised O, 256- or
 // 512-byte rows, so each starts on an L2 line) and, separately, one float l
@@ -49,9 +51,10 @@ inline int bucket_lead(long long rows_per_kv_head, int row_bytes) {
   return (int)(n < 0 ? 0 : (n > 2 ? 2 : n));
 }
 
+// cent_norm_max: each KV head's largest centroid 2-norm (launch_conv_centroid).
 cudaError_t launch_route(const bf16* q, const bf16* k, const bf16* cent_hi, const bf16* cent_lo,
-                         const SeqPlan& p, int h_q, int h_kv, int d, int block_size, int topk,
-                         int32_t* sel_idx, float* mref, int32_t* flag, float* oacc, float* lacc,
+                         const float* cent_norm_max, const SeqPlan& p, int h_q, int h_kv, int d, int block_size,
+                         int topk, int32_t* sel_idx, float* mref, int32_t* flag, float* oacc, float* lacc,
                          int32_t* status, cudaStream_t st);
 
 // chunk_cnt (optional, index_chunk_ints() int32) selects the shared-memory

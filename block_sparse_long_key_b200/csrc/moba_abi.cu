@@ -65,6 +65,7 @@ struct FwdBufs {
   float* cent;
   bf16* hi;
   bf16* lo;
+  float* cnorm;  // largest centroid norm per KV head (router screen margin)
   float* mref;
   int32_t* flag;
   float* oacc;  // rows of oacc_stride(d) floats: the unnormalised O
@@ -86,6 +87,7 @@ FwdBufs carve_fwd(Carve& c, const moba_shape* s) {
   b.cent = c.take<float>(ncent);
   b.hi = c.take<bf16>(ncent);
   b.lo = c.take<bf16>(ncent);
+  b.cnorm = c.take<float>(s->h_kv);
   b.mref = c.take<float>(nrow);
   b.flag = c.take<int32_t>(nrow);
   b.oacc = c.take<float>(nrow * moba::oacc_stride(s->head_dim));
@@ -221,7 +223,7 @@ int moba_key_conv_centroid(const void* k, const float* conv_w, int conv_width, c
   if ((rc = begin_plan(b.plan, cu_seqlens, shape, st, &plan, -1)) != MOBA_OK) return rc;
   MOBA_TRY(moba::launch_conv_centroid(static_cast<const bf16*>(k), conv_w, conv_width, plan, shape->h_kv,
                                       shape->head_dim, shape->block_size, static_cast<bf16*>(k_out), centroid, b.hi,
-                                      b.lo, st));
+                                      b.lo, nullptr, st));
   return MOBA_OK;
 }
 
@@ -247,12 +249,13 @@ int moba_forward(const void* q, const void* k, const void* v, const int32_t* cu_
   const bf16* kk = conv_width > 0 ? static_cast<const bf16*>(k_conv_out) : static_cast<const bf16*>(k);
   const bf16* kv = static_cast<const bf16*>(v);
   STAGE_BEGIN(MOBA_STAGE_FWD_CENTROID);
+  MOBA_TRY(cudaMemsetAsync(b.cnorm, 0, sizeof(float) * hkv, st));
   MOBA_TRY(moba::launch_conv_centroid(static_cast<const bf16*>(k), conv_w, conv_width, plan, hkv, d, B,
-                                      static_cast<bf16*>(k_conv_out), b.cent, b.hi, b.lo, st));
+                                      static_cast<bf16*>(k_conv_out), b.cent, b.hi, b.lo, b.cnorm, st));
   STAGE_END(MOBA_STAGE_FWD_CENTROID);
   STAGE_BEGIN(MOBA_STAGE_FWD_ROUTE);
-  MOBA_TRY(moba::launch_route(kq, kk, b.hi, b.lo, plan, hq, hkv, d, B, topk, sel_idx, b.mref, b.flag, b.oacc, b.lacc,
-                              b.plan.status, st));
+  MOBA_TRY(moba::launch_route(kq, kk, b.hi, b.lo, b.cnorm, plan, hq, hkv, d, B, topk, sel_idx, b.mref, b.flag, b.oacc,
+                              b.lacc, b.plan.status, st));
   STAGE_END(MOBA_STAGE_FWD_ROUTE);
   STAGE_BEGIN(MOBA_STAGE_FWD_INDEX);
   MOBA_TRY(moba::launch_build_index(sel_idx, plan, hq, hkv, B, topk, b.cnt, b.ptr, b.cursor, b.rows,

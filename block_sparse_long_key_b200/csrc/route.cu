@@ -134,7 +134,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
              const int32_t* __restrict__ blk_off, const int32_t* __restrict__ tile_off, int batch,
              int nb_max, int h_q, int h_kv, int block_size, int topk, int32_t* __restrict__ sel_idx,
              float* __restrict__ mref, int32_t* __restrict__ flag, float* __restrict__ oacc, float* __restrict__ lacc,
-             int32_t* __restrict__ status) {
+             const float* __restrict__ cent_norm_max, int32_t* __restrict__ status) {
   using Ly = RouteLayout<D, NC, LISTN>;
   // Sift depth of a complete tree with LISTN - 1 nodes (children of the
   // deepest internal node still lie below LISTN - 1).
@@ -183,13 +183,14 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   // NC rows x 64 values; rows past `nscan` (the next sequence's or head's
   // blocks, or beyond the table: zero) are scored but never selected.
   const int crow0 = kvh * nb_max + cbase;
-  auto load_chunk = [&](int c, int buf) {
-    tc::mbar_arrive_expect_tx(mb_c0 + 8 * buf, 2 * Ly::C_MAT);
+  // The screen pass (step < nchunks of a two-pass tile) needs only the hi halves.
+  auto load_chunk = [&](int c, int buf, bool hi_only) {
+    tc::mbar_arrive_expect_tx(mb_c0 + 8 * buf, (hi_only ? 1 : 2) * Ly::C_MAT);
 #pragma unroll
     for (int r = 0; r < Ly::KB; ++r) {
       const uint32_t dst = sbase + Ly::C_OFF + buf * Ly::C_BUF + r * Ly::C_REGION;
       tc::tma_load_2d(dst, &tm_hi, r * 64, crow0 + c * NC, mb_c0 + 8 * buf);
-      tc::tma_load_2d(dst + Ly::C_MAT, &tm_lo, r * 64, crow0 + c * NC, mb_c0 + 8 * buf);
+      if (!hi_only) tc::tma_load_2d(dst + Ly::C_MAT, &tm_lo, r * 64, crow0 + c * NC, mb_c0 + 8 * buf);
     }
   };
 
@@ -232,20 +233,26 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   __syncthreads();
   tc::fence_after_sync();
   const bool producer = tid == kSel;  // lane 0 of the last warp
+  auto screen_step = [&](int st) { return two_pass && st < nchunks; };
   if (producer)
-    for (int b = 0; b < Ly::kCB && b < nsteps; ++b) load_chunk(chunk_of(b), b);
+    for (int b = 0; b < Ly::kCB && b < nsteps; ++b) load_chunk(chunk_of(b), b, screen_step(b));
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Ly::HOLD_OFF);
   constexpr uint32_t idesc = tc::idesc_bf16_f32(kTM, NC);
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  float qn2 = 0.f;  // |q|^2 of the thread's row
   if (nchunks > 0 && sel_thread) {
     // Q row `tid` -> TMEM lane `tid`, columns TM_Q .. TM_Q + D/2 (bf16 pairs).
     const bf16* qrow = q + (size_t)(t0 + tid) * qstride + (size_t)h * D;
 #pragma unroll
     for (int half = 0; half < D / 64; ++half) {
-      uint32_t w[32];
+      uint32_t w[32];  // (the row's squared norm accumulates in qn2 on the way)
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const uint4 u = row_ok ? __ldg(reinterpret_cast<const uint4*>(qrow + half * 64 + c * 8)) : make_uint4(0, 0, 0, 0);
+        float f[8];
+        bf16x8_to_f32(u, f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qn2 = fmaf(f[i], f[i], qn2);
         w[4 * c] = u.x;
         w[4 * c + 1] = u.y;
         w[4 * c + 2] = u.z;
@@ -382,7 +389,7 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
         // chunk c - 1's MMAs are done with its buffer: load chunk c + kCB - 1 there
         const int pc = c - 1;
         if (!(ok = tc::mbar_wait(mb_full + 8 * (pc % Ly::NB), (pc / Ly::NB) & 1))) break;
-        load_chunk(chunk_of(c + Ly::kCB - 1), pc % Ly::kCB);
+        load_chunk(chunk_of(c + Ly::kCB - 1), pc % Ly::kCB, screen_step(c + Ly::kCB - 1));
       }
       if (!(ok = tc::mbar_wait(mb_c0 + 8 * buf, (c / Ly::kCB) & 1))) break;
       if (c >= Ly::NB && !(ok = tc::mbar_wait(mb_empty + 8 * sc, ((c / Ly::NB) - 1) & 1))) break;
@@ -395,11 +402,13 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
         const uint32_t koff = (kk & 3) * 32;  // 16 bf16 per K step inside a 128-byte row
         tc::mma_bf16_ts(d_tmem, qa + kk * 8, tc::sw128_desc(ca + (kk >> 2) * Ly::C_REGION + koff), idesc, kk > 0);
       }
+      if (!screen_step(c)) {
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t koff = (kk & 3) * 32;
-        tc::mma_bf16_ts(d_tmem, qa + kk * 8, tc::sw128_desc(ca + Ly::C_MAT + (kk >> 2) * Ly::C_REGION + koff), idesc,
-                        1u);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk & 3) * 32;
+          tc::mma_bf16_ts(d_tmem, qa + kk * 8, tc::sw128_desc(ca + Ly::C_MAT + (kk >> 2) * Ly::C_REGION + koff),
+                          idesc, 1u);
+        }
       }
       tc::mma_commit(mb_full + 8 * sc);
     }
@@ -466,6 +475,14 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
       lb = INFINITY;
 #pragma unroll
       for (int i = 0; i < kBoundList; ++i) lb = i < k2 ? fminf(lb, top2[i]) : lb;
+      // The screen scored q . c_hi; the exact score adds q . c_lo and its
+      // fp32 rounding.  |q . c_lo| <= |q| |c_lo| <= 2^-9 (1 + 2^-9) |q| |c|
+      // (c_lo is c - c_hi rounded to bf16), and the added accumulation steps
+      // round far below 2^-14 |q| |c|: lowering the bound by
+      // E = |q| max_j |c_j| (2^-9 + 2^-14), rounded down, keeps it below the
+      // exact scores of the k - 1 blocks that reached it in the screen.
+      const float err = sqrtf(qn2) * __ldg(cent_norm_max + kvh) * (0.001953125f + 0.00006103515625f) * 1.0001f;
+      lb = __fsub_rd(lb, err);
       thr = fmaxf(tau, nextafterf(lb, -INFINITY));
     }
     // (Second) pass: selection into the heap.
@@ -553,8 +570,8 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
 }
 
 template <int D, int NC, int LISTN>
-cudaError_t launch_route_t(const bf16* q, const bf16* k, const bf16* hi, const bf16* lo, const SeqPlan& p,
-                           int h_q, int h_kv, int block_size, int topk, int32_t* sel, float* mref,
+cudaError_t launch_route_t(const bf16* q, const bf16* k, const bf16* hi, const bf16* lo, const float* cnorm,
+                           const SeqPlan& p, int h_q, int h_kv, int block_size, int topk, int32_t* sel, float* mref,
                            int32_t* flag, float* oacc, float* lacc, int32_t* status, cudaStream_t st) {
   const size_t smem = RouteLayout<D, NC, LISTN>::BYTES + 1024;
   auto kern = route_kernel<D, NC, LISTN>;
@@ -570,18 +587,19 @@ cudaError_t launch_route_t(const bf16* q, const bf16* k, const bf16* hi, const b
   if (e != cudaSuccess) return e;
   dim3 grid(max_tiles * h_q);
   kern<<<grid, kThreads, smem, st>>>(q, k, tm_hi, tm_lo, p.cu, p.blk_off, p.tile_off, p.batch, p.nb_max, h_q,
-                                     h_kv, block_size, topk, sel, mref, flag, oacc, lacc, status);
+                                     h_kv, block_size, topk, sel, mref, flag, oacc, lacc, cnorm, status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_route(const bf16* q, const bf16* k, const bf16* hi, const bf16* lo, const SeqPlan& p,
-                         int h_q, int h_kv, int d, int block_size, int topk, int32_t* sel, float* mref,
-                         int32_t* flag, float* oacc, float* lacc, int32_t* status, cudaStream_t st) {
+cudaError_t launch_route(const bf16* q, const bf16* k, const bf16* hi, const bf16* lo, const float* cnorm,
+                         const SeqPlan& p, int h_q, int h_kv, int d, int block_size, int topk, int32_t* sel,
+                         float* mref, int32_t* flag, float* oacc, float* lacc, int32_t* status, cudaStream_t st) {
   const int k1 = topk - 1;
 #define MOBA_ROUTE(DD, NCC, LN) \
-  return launch_route_t<DD, NCC, LN>(q, k, hi, lo, p, h_q, h_kv, block_size, topk, sel, mref, flag, oacc, lacc, status, st)
+  return launch_route_t<DD, NCC, LN>(q, k, hi, lo, cnorm, p, h_q, h_kv, block_size, topk, sel, mref, flag, oacc, lacc, \
+                                     status, st)
   if (d == 64) {
     if (k1 <= 32) MOBA_ROUTE(64, 32, 32);
     MOBA_ROUTE(64, 32, 64);
