@@ -25,6 +25,7 @@ SMALL = [
     ((900,), 2, 2, 64, 32, 1, 0),                   # topk=1: block-diagonal causal
     ((600,), 1, 1, 128, 32, 64, 0),                 # topk=64 >= n: dense causal
     ((3000,), 8, 2, 64, 64, 16, 3),                 # GQA 4:1, conv width 3
+    ((2500, 77), 4, 1, 64, 16, 6, 0),               # GQA 4:1, B=16: buckets of many 128-row tiles
 ]
 
 
