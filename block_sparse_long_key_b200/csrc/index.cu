@@ -135,11 +135,11 @@ fill_kernel(const int32_t* __restrict__ sel_idx, long long npicks, int topk, int
 
 // ---- shared-memory privatised path
 //
-// A CTA owns the picks of one (chunk of kChunkTokens tokens, KV head): one
-// thread per query row (token, query head of the group) at a time, which
-// locates its sequence once and then walks the row's topk picks (16-byte
-// loads), so the per-pick work is a load, a range check and one
-// shared-memory atomic.
+// A CTA owns the picks of one (chunk of kChunkTokens tokens, KV head).  The
+// count and the staged fill take one pick per thread and step (coalesced
+// loads, several independent picks in flight per thread); the unstaged fill
+// takes one query row per thread and walks its topk picks.  The per-pick
+// work is a load, a range check and one shared-memory atomic.
 
 // For query row `r` of the chunk (ta: first token): its row id, its
 // sequence's first global block and its own block; false past the chunk or
@@ -185,25 +185,83 @@ __device__ __forceinline__ void for_row_picks(const int32_t* __restrict__ sel_id
   for (; m < topk; ++m) one(m, __ldg(p + m));
 }
 
-__global__ void __launch_bounds__(kThreads)
+// Threads of the per-chunk count and staged fill.  A thread takes a run of
+// kRun consecutive slots of one query row (two 16-byte loads when topk is a
+// multiple of 4), so the row's sequence is located once per run and a warp's
+// loads of sel_idx are contiguous; a CTA covers kPickThreads runs per step.
+constexpr int kPickThreads = 1024;
+constexpr int kRun = 8;
+
+// Run q of a chunk (rpr = ceil(topk / kRun) runs per query row): slots
+// [m0, m0 + kRun) of chunk row r = q / rpr.  Sets `row` and bk[i] to the
+// block offset of slot m0 + i in the KV head's histogram (sequence base +
+// block), or -1 for a slot past topk, an empty or invalid slot (invalid ones
+// raise kStatusBadSelIdx when `kReport`) or a row outside every sequence.
+template <bool kReport>
+__device__ __forceinline__ void chunk_run(const int32_t* __restrict__ sel_idx, int q, int rpr, int topk, int ntok,
+                                          int ta, int kvh, int group, int h_q, int block_size, const int32_t* cu,
+                                          const int32_t* blk_off, int batch, int seq_end, int32_t* status, int& row,
+                                          int (&bk)[kRun]) {
+  const int r = q / rpr, m0 = (q - r * rpr) * kRun;
+  int bb, own;
+#pragma unroll
+  for (int i = 0; i < kRun; ++i) bk[i] = -1;
+  if (!chunk_row(r, ntok, ta, kvh, group, h_q, block_size, cu, blk_off, batch, seq_end, row, bb, own)) return;
+  const int32_t* src = sel_idx + (size_t)row * topk + m0;
+  int j[kRun];
+  if ((topk & 3) == 0) {  // 16-byte aligned: m0 is a multiple of 8, row * topk of 4
+#pragma unroll
+    for (int i = 0; i < kRun; i += 4) {
+      if (m0 + i < topk) {
+        const int4 v = __ldg(reinterpret_cast<const int4*>(src + i));
+        j[i] = v.x;
+        j[i + 1] = v.y;
+        j[i + 2] = v.z;
+        j[i + 3] = v.w;
+      } else {
+        j[i] = j[i + 1] = j[i + 2] = j[i + 3] = -1;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kRun; ++i) j[i] = m0 + i < topk ? __ldg(src + i) : -1;
+  }
+#pragma unroll
+  for (int i = 0; i < kRun; ++i) {
+    if (j[i] < 0) {
+      if (kReport && j[i] != -1) set_status(status, kStatusBadSelIdx);
+    } else if (j[i] > own) {
+      if (kReport) set_status(status, kStatusBadSelIdx);
+    } else {
+      bk[i] = bb + j[i];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kPickThreads)
 chunk_count_kernel(const int32_t* __restrict__ sel_idx, int total_tokens, int topk, int h_q, int group,
                    int block_size, const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off, int batch,
                    int nb_max, int nchunks, int32_t* __restrict__ chunk_cnt, int32_t* __restrict__ status) {
   extern __shared__ int32_t hist[];
-  const int c = blockIdx.x, kvh = blockIdx.y;
-  for (int b = threadIdx.x; b < nb_max; b += kThreads) hist[b] = 0;
+  const int c = blockIdx.x, kvh = blockIdx.y, tid = threadIdx.x;
+  for (int b = tid; b < nb_max; b += kPickThreads) hist[b] = 0;
   __syncthreads();
   const int ta = c * kChunkTokens;
   const int ntok = max(0, min(kChunkTokens, total_tokens - ta));
   const int seq_end = __ldg(cu + batch);
-  for (int r = threadIdx.x; r < ntok * group; r += kThreads) {
-    int row, base, own;
-    if (!chunk_row(r, ntok, ta, kvh, group, h_q, block_size, cu, blk_off, batch, seq_end, row, base, own)) continue;
-    for_row_picks<true>(sel_idx, row, topk, own, status, [&](int, int j) { atomicAdd(hist + base + j, 1); });
+  const int rpr = (topk + kRun - 1) / kRun;
+  const int nruns = ntok * group * rpr;
+  for (int q = tid; q < nruns; q += kPickThreads) {
+    int row, bk[kRun];
+    chunk_run<true>(sel_idx, q, rpr, topk, ntok, ta, kvh, group, h_q, block_size, cu, blk_off, batch, seq_end, status,
+                    row, bk);
+#pragma unroll
+    for (int i = 0; i < kRun; ++i)
+      if (bk[i] >= 0) atomicAdd(hist + bk[i], 1);
   }
   __syncthreads();
   int32_t* dst = chunk_cnt + ((size_t)kvh * nchunks + c) * nb_max;
-  for (int b = threadIdx.x; b < nb_max; b += kThreads) dst[b] = hist[b];
+  for (int b = tid; b < nb_max; b += kPickThreads) dst[b] = hist[b];
 }
 
 // Per bucket: chunk counts -> exclusive prefix over chunks (in place), total
@@ -253,26 +311,28 @@ chunk_fill_kernel(const int32_t* __restrict__ sel_idx, int total_tokens, int top
   }
 }
 
-// Staged fill (blocks per KV head <= kMaxStagedBuckets): the chunk's rows are
-// taken in passes of at most kStage picks.  A pass counts its picks per block
-// in shared memory, scans the counts into local bucket starts, places each
-// row id at its local slot (with its bucket as a tag) and then copies the
-// staged entries out in order: consecutive entries of one bucket go to
-// consecutive addresses, so the stores coalesce into runs instead of one
-// scattered 4-byte store per pick.  `base[b]` is where the chunk's next entry
-// for block b goes in rows[].
-constexpr int kStage = 8192;
+// Staged fill (blocks per KV head <= kMaxStagedBuckets): the chunk's runs
+// are taken in passes of kPickThreads, one per thread (at most kStage
+// picks).  A pass counts its picks per block in shared memory, scans the counts
+// into local bucket starts, places each row id at its local slot (with its
+// bucket as a tag; the picks' buckets stay in registers between the two
+// steps) and then copies the staged entries out in order: consecutive
+// entries of one bucket go to consecutive addresses, so the stores coalesce
+// into runs instead of one scattered 4-byte store per pick.  `base[b]` is
+// where the chunk's next entry for block b goes in rows[].
+constexpr int kStage = kPickThreads * kRun;
 constexpr int kMaxStagedBuckets = 8192;
 
 __host__ __device__ constexpr size_t staged_fill_smem(int nb_max) {
   return sizeof(int32_t) * (2 * (size_t)nb_max + 1 + kStage) + sizeof(uint16_t) * kStage;
 }
 
-// In-place exclusive scan of a[0..n) by the whole CTA (kThreads threads);
-// returns the total.  `part` holds kThreads ints of shared scratch.
+// In-place exclusive scan of a[0..n) by the whole CTA (NT threads, NT <=
+// 1024); returns the total.  `part` holds NT / 32 + 1 ints of shared scratch.
+template <int NT>
 __device__ int block_exclusive_scan(int32_t* a, int n, int32_t* part) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (n + kThreads - 1) / kThreads;
+  const int per = (n + NT - 1) / NT;
   const int lo = min(tid * per, n), hi = min(lo + per, n);
   int sum = 0;
   for (int i = lo; i < hi; ++i) sum += a[i];
@@ -285,15 +345,15 @@ __device__ int block_exclusive_scan(int32_t* a, int n, int32_t* part) {
   if (lane == 31) part[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const int v = lane < kThreads / 32 ? part[lane] : 0;
+    const int v = lane < NT / 32 ? part[lane] : 0;
     int w = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int o = __shfl_up_sync(0xffffffffu, w, off);
       if (lane >= off) w += o;
     }
-    if (lane < kThreads / 32) part[lane] = w - v;
-    if (lane == 31) part[kThreads / 32] = w;  // total
+    if (lane < NT / 32) part[lane] = w - v;
+    if (lane == 31) part[NT / 32] = w;  // total
   }
   __syncthreads();
   int run = part[warp] + incl - sum;
@@ -302,12 +362,12 @@ __device__ int block_exclusive_scan(int32_t* a, int n, int32_t* part) {
     a[i] = run;
     run += v;
   }
-  const int total = part[kThreads / 32];
+  const int total = part[NT / 32];
   __syncthreads();
   return total;
 }
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kPickThreads, 2)
 chunk_fill_staged_kernel(const int32_t* __restrict__ sel_idx, int total_tokens, int topk, int h_q, int group,
                          int block_size, const int32_t* __restrict__ cu, const int32_t* __restrict__ blk_off,
                          int batch, int nb_max, int nchunks, const int32_t* __restrict__ chunk_cnt,
@@ -317,51 +377,54 @@ chunk_fill_staged_kernel(const int32_t* __restrict__ sel_idx, int total_tokens, 
   int32_t* lc = base + nb_max;              // [nb_max + 1]: counts -> local starts -> cursors
   int32_t* stage = lc + nb_max + 1;         // [kStage]
   uint16_t* tag = reinterpret_cast<uint16_t*>(stage + kStage);  // [kStage]
-  __shared__ int32_t part[kThreads / 32 + 1];
+  __shared__ int32_t part[kPickThreads / 32 + 1];
   const int c = blockIdx.x, kvh = blockIdx.y;
   const int tid = threadIdx.x;
   const int32_t* src = chunk_cnt + ((size_t)kvh * nchunks + c) * nb_max;
   const int32_t* bptr = ptr + (size_t)kvh * nb_max;
-  for (int b = tid; b < nb_max; b += kThreads) base[b] = __ldg(bptr + b) + __ldg(src + b);
+  for (int b = tid; b < nb_max; b += kPickThreads) base[b] = __ldg(bptr + b) + __ldg(src + b);
   const int ta = c * kChunkTokens;
   const int ntok = max(0, min(kChunkTokens, total_tokens - ta));
   const int seq_end = __ldg(cu + batch);
-  const int nrows = ntok * group;
-  const int pass_rows = max(1, kStage / topk);
-  for (int r0 = 0; r0 < nrows; r0 += pass_rows) {
-    const int r1 = min(nrows, r0 + pass_rows);
-    for (int b = tid; b <= nb_max; b += kThreads) lc[b] = 0;
+  const int rpr = (topk + kRun - 1) / kRun;
+  const int nruns = ntok * group * rpr;
+  for (int q0 = 0; q0 < nruns; q0 += kPickThreads) {
+    for (int b = tid; b <= nb_max; b += kPickThreads) lc[b] = 0;
     __syncthreads();
-    // 1. count this pass's picks per block (invalid entries were reported by
-    //    the count pass and are skipped here)
-    for (int r = r0 + tid; r < r1; r += kThreads) {
-      int row, bb, own;
-      if (!chunk_row(r, ntok, ta, kvh, group, h_q, block_size, cu, blk_off, batch, seq_end, row, bb, own)) continue;
-      for_row_picks<false>(sel_idx, row, topk, own, nullptr, [&](int, int j) { atomicAdd(lc + bb + j, 1); });
+    // 1. this pass's runs: bucket offsets (invalid entries were reported by
+    //    the count pass and are skipped here), counted per block
+    int row = 0, bk[kRun];
+    if (q0 + tid < nruns) {
+      chunk_run<false>(sel_idx, q0 + tid, rpr, topk, ntok, ta, kvh, group, h_q, block_size, cu, blk_off, batch,
+                       seq_end, nullptr, row, bk);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kRun; ++i) bk[i] = -1;
     }
+#pragma unroll
+    for (int i = 0; i < kRun; ++i)
+      if (bk[i] >= 0) atomicAdd(lc + bk[i], 1);
     __syncthreads();
     // 2. local bucket starts
-    const int total = block_exclusive_scan(lc, nb_max, part);
+    const int total = block_exclusive_scan<kPickThreads>(lc, nb_max, part);
     // 3. stage each row id at its local slot
-    for (int r = r0 + tid; r < r1; r += kThreads) {
-      int row, bb, own;
-      if (!chunk_row(r, ntok, ta, kvh, group, h_q, block_size, cu, blk_off, batch, seq_end, row, bb, own)) continue;
-      for_row_picks<false>(sel_idx, row, topk, own, nullptr, [&](int, int j) {
-        const int slot = atomicAdd(lc + bb + j, 1);
-        stage[slot] = row;
-        tag[slot] = (uint16_t)(bb + j);
-      });
+#pragma unroll
+    for (int i = 0; i < kRun; ++i) {
+      if (bk[i] < 0) continue;
+      const int slot = atomicAdd(lc + bk[i], 1);
+      stage[slot] = row;
+      tag[slot] = (uint16_t)bk[i];
     }
     __syncthreads();
     // 4. copy out in order; lc[b] is now the end of bucket b's local run, so
     //    the run starts at lc[b - 1]
-    for (int i = tid; i < total; i += kThreads) {
+    for (int i = tid; i < total; i += kPickThreads) {
       const int b = tag[i];
       const int start = b > 0 ? lc[b - 1] : 0;
       rows[base[b] + (i - start)] = stage[i];
     }
     __syncthreads();
-    for (int b = tid; b < nb_max; b += kThreads) base[b] += lc[b] - (b > 0 ? lc[b - 1] : 0);
+    for (int b = tid; b < nb_max; b += kPickThreads) base[b] += lc[b] - (b > 0 ? lc[b - 1] : 0);
     __syncthreads();
   }
 }
@@ -391,7 +454,7 @@ cudaError_t launch_build_index(const int32_t* sel_idx, const SeqPlan& p, int h_q
         cudaSuccess)
       return e;
     dim3 grid(nchunks, h_kv);
-    chunk_count_kernel<<<grid, kThreads, smem, st>>>(sel_idx, p.total_tokens, topk, h_q, group, block_size, p.cu,
+    chunk_count_kernel<<<grid, kPickThreads, smem, st>>>(sel_idx, p.total_tokens, topk, h_q, group, block_size, p.cu,
                                                      p.blk_off, p.batch, p.nb_max, nchunks, chunk_cnt, status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     chunk_prefix_kernel<<<(nbk + kThreads - 1) / kThreads, kThreads, 0, st>>>(chunk_cnt, p.nb_max, nchunks, h_kv,
@@ -404,7 +467,7 @@ cudaError_t launch_build_index(const int32_t* sel_idx, const SeqPlan& p, int h_q
       if ((e = cudaFuncSetAttribute(chunk_fill_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)smem2)) != cudaSuccess)
         return e;
-      chunk_fill_staged_kernel<<<grid, kThreads, smem2, st>>>(sel_idx, p.total_tokens, topk, h_q, group, block_size,
+      chunk_fill_staged_kernel<<<grid, kPickThreads, smem2, st>>>(sel_idx, p.total_tokens, topk, h_q, group, block_size,
                                                               p.cu, p.blk_off, p.batch, p.nb_max, nchunks, chunk_cnt,
                                                               ptr, rows);
       return cudaGetLastError();
