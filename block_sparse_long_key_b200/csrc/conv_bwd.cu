@@ -82,41 +82,49 @@ conv_bwd_kernel(const bf16* __restrict__ k, const float* __restrict__ conv_w, co
   cp_async_wait<0>();
   __syncthreads();
 
-  // kwin[l] = k_{u-l}; pend[l] accumulates sum_m W_m g_{t+m} for t = u - l;
-  // dwa[l] = sum over the block's u of g_u k_{u-l}.
-  float kwin[W], pend[W], dwa[W];
+  // Register rings indexed by the step's residue mod W, which is a
+  // compile-time constant inside the unrolled inner loop, so no value moves
+  // between registers as u advances: kr[(r - l) % W] = k_{u-l},
+  // gr[r % W] = dK'_u, pr[(r - l) % W] accumulates sum_m W_m g_{t+m} for
+  // t = u - l (the slot of t = u - (W - 1) is emitted at step r and taken by
+  // t = u + 1 at the next); dwa[l] = sum over the block's u of g_u k_{u-l}.
+  constexpr int R = BLK + W - 1;  // steps u = t0 + r, r < R
+  float kr[W], gr[W], pr[W], dwa[W];
 #pragma unroll
-  for (int l = 0; l < W; ++l) {
-    pend[l] = dwa[l] = 0.f;
-    kwin[l] = l >= 1 ? __bfloat162float(ks[(W - 1 - l) * Ly::SEG + ch]) : 0.f;
-  }
+  for (int l = 0; l < W; ++l) kr[l] = gr[l] = pr[l] = dwa[l] = 0.f;
+#pragma unroll
+  for (int l = 1; l < W; ++l) kr[W - l] = __bfloat162float(ks[(W - 1 - l) * Ly::SEG + ch]);  // k_{t0-l}
   const int n = t1 - t0;
-#pragma unroll 2
-  for (int r = 0; r < BLK + W - 1; ++r) {  // u = t0 + r
-    kwin[0] = __bfloat162float(ks[(W - 1 + r) * Ly::SEG + ch]);
-    float g = 0.f;
-    if (t0 + r < seq1) {
-      float x = 0.f;
+  for (int r0 = 0; r0 < R; r0 += W) {
 #pragma unroll
-      for (int l = 0; l < W; ++l) x = fmaf(w[l], kwin[l], x);
-      const float sg = __frcp_rn(1.f + __expf(-x));
-      g = __bfloat162float(gs[r * Ly::SEG + ch]) * sg * (1.f + x * (1.f - sg));
+    for (int i = 0; i < W; ++i) {
+      const int r = r0 + i;
+      if (r < R) {
+        kr[i] = __bfloat162float(ks[(W - 1 + r) * Ly::SEG + ch]);
+        gr[i] = __bfloat162float(gs[r * Ly::SEG + ch]);
+        float g = 0.f;
+        if (t0 + r < seq1) {
+          float x = 0.f;
+#pragma unroll
+          for (int l = 0; l < W; ++l) x = fmaf(w[l], kr[(i - l + W) % W], x);
+          const float sg = __fdividef(1.f, 1.f + __expf(-x));
+          g = gr[i] * sg * (1.f + x * (1.f - sg));
+        }
+        if (r < n) {
+#pragma unroll
+          for (int l = 0; l < W; ++l) dwa[l] = fmaf(g, kr[(i - l + W) % W], dwa[l]);
+        }
+        // t = u takes its first term here: assigning it also drops what the
+        // first W - 1 steps added to this slot for tokens before the block
+        pr[i] = w[0] * g;
+#pragma unroll
+        for (int l = 1; l < W; ++l) pr[(i - l + W) % W] = fmaf(w[l], g, pr[(i - l + W) % W]);
+        if (r >= W - 1) {  // t = u - (W - 1) is complete (slot (i + 1) % W)
+          const int sl = (i + 1) % W;
+          os[(r - (W - 1)) * Ly::SEG + ch] = __float2bfloat16_rn(gr[sl] + pr[sl]);
+        }
+      }
     }
-    if (r < n) {
-#pragma unroll
-      for (int l = 0; l < W; ++l) dwa[l] = fmaf(g, kwin[l], dwa[l]);
-    }
-#pragma unroll
-    for (int l = 0; l < W; ++l) pend[l] = fmaf(w[l], g, pend[l]);
-    const int te = r - (W - 1);  // t = t0 + te is complete now
-    if (te >= 0 && te < BLK)
-      os[te * Ly::SEG + ch] = __float2bfloat16_rn(__bfloat162float(gs[te * Ly::SEG + ch]) + pend[W - 1]);
-#pragma unroll
-    for (int l = W - 1; l > 0; --l) {
-      kwin[l] = kwin[l - 1];
-      pend[l] = pend[l - 1];
-    }
-    pend[0] = 0.f;
   }
   __syncthreads();
   for (int i = tid; i < n * CPR; i += kThreads) {
@@ -132,23 +140,33 @@ conv_bwd_kernel(const bf16* __restrict__ k, const float* __restrict__ conv_w, co
   }
 }
 
-// dW[h][c][l] = sum over the blocks of head h: one warp per output, lane i
-// sums blocks i, i+32, ..., then a fixed shuffle tree (deterministic).
-__global__ void __launch_bounds__(kThreads)
+// dW[h][c][l] = sum over the blocks of head h.  One CTA per (head, 32
+// consecutive (channel, tap) entries): lane i of warp w sums entry i over
+// blocks w, w + 32, ... (each warp load is one 128-byte row piece), then
+// warp 0 adds the 32 warp sums in a fixed order (deterministic).
+constexpr int kDwThreads = 1024;
+__global__ void __launch_bounds__(kDwThreads)
 conv_dw_reduce_kernel(const float* __restrict__ dw_part, const int32_t* __restrict__ blk_off, int batch, int nb_max,
-                      int h_kv, int dwid, float* __restrict__ dw) {
-  const int i = (blockIdx.x * kThreads + threadIdx.x) >> 5;  // over h_kv * dwid
-  const int lane = threadIdx.x & 31;
-  if (i >= h_kv * dwid) return;
-  const int h = i / dwid, cl = i % dwid;
+                      int dwid, float* __restrict__ dw) {
+  __shared__ float part[32][33];
+  const int groups = (dwid + 31) / 32;
+  const int h = blockIdx.x / groups, cl = (blockIdx.x % groups) * 32 + (threadIdx.x & 31);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nb = __ldg(blk_off + batch);
   const float* src = dw_part + (size_t)h * nb_max * dwid + cl;
   float acc = 0.f;
+  if (cl < dwid) {
 #pragma unroll 4
-  for (int b = lane; b < nb; b += 32) acc += __ldg(src + (size_t)b * dwid);
+    for (int b = warp; b < nb; b += 32) acc += __ldg(src + (size_t)b * dwid);
+  }
+  part[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0 && cl < dwid) {
+    float t = 0.f;
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) dw[i] = acc;
+    for (int w2 = 0; w2 < 32; ++w2) t += part[w2][lane];
+    dw[(size_t)h * dwid + cl] = t;
+  }
 }
 
 template <int D, int W>
@@ -175,9 +193,8 @@ cudaError_t launch_conv_bwd_t(const bf16* k, const float* conv_w, const bf16* dk
   }
 #undef MOBA_CB
   if (e != cudaSuccess) return e;
-  const long long nthreads = (long long)h_kv * D * W * 32;
-  conv_dw_reduce_kernel<<<(int)((nthreads + kThreads - 1) / kThreads), kThreads, 0, st>>>(dw_part, p.blk_off, p.batch,
-                                                                                         p.nb_max, h_kv, D * W, dw);
+  const int groups = (D * W + 31) / 32;
+  conv_dw_reduce_kernel<<<h_kv * groups, kDwThreads, 0, st>>>(dw_part, p.blk_off, p.batch, p.nb_max, D * W, dw);
   return cudaGetLastError();
 }
 

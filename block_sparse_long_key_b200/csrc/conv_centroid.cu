@@ -83,22 +83,28 @@ conv_centroid_kernel(const bf16* __restrict__ k, const float* __restrict__ conv_
   if constexpr (W == 0) {
     for (int r = 0; r < n; ++r) acc += __bfloat162float(in[r * Ly::SEG + ch]);
   } else {
-    // win[l] = k_{t-1-l}
-    float win[W > 1 ? W - 1 : 1];
+    // Register ring indexed by the row's residue mod W (a compile-time
+    // constant inside the unrolled inner loop, so no value moves as t
+    // advances): kr[(r - l) % W] = k_{t-l} for t = t0 + r.
+    float kr[W];
 #pragma unroll
-    for (int l = 0; l < W - 1; ++l) win[l] = __bfloat162float(in[(Ly::PRE - 1 - l) * Ly::SEG + ch]);
-#pragma unroll 4
-    for (int r = 0; r < BLK; ++r) {
-      const float cur = __bfloat162float(in[(Ly::PRE + r) * Ly::SEG + ch]);
-      float x = w[0] * cur;
+    for (int l = 0; l < W; ++l) kr[l] = 0.f;
 #pragma unroll
-      for (int l = 1; l < W; ++l) x = fmaf(w[l], win[l - 1], x);
-      const bf16 y = __float2bfloat16_rn(cur + __fdividef(x, 1.f + __expf(-x)));  // k + SiLU(x)
-      outt[r * Ly::SEG + ch] = y;
-      if (r < n) acc += __bfloat162float(y);  // the centroid averages the stored bf16 keys
+    for (int l = 1; l < W; ++l) kr[W - l] = __bfloat162float(in[(Ly::PRE - l) * Ly::SEG + ch]);  // k_{t0-l}
+    for (int r0 = 0; r0 < BLK; r0 += W) {
 #pragma unroll
-      for (int l = W - 2; l > 0; --l) win[l] = win[l - 1];
-      if (W > 1) win[0] = cur;
+      for (int i = 0; i < W; ++i) {
+        const int r = r0 + i;
+        if (r < BLK) {
+          kr[i] = __bfloat162float(in[(Ly::PRE + r) * Ly::SEG + ch]);
+          float x = 0.f;
+#pragma unroll
+          for (int l = 0; l < W; ++l) x = fmaf(w[l], kr[(i - l + W) % W], x);
+          const bf16 y = __float2bfloat16_rn(kr[i] + __fdividef(x, 1.f + __expf(-x)));  // k + SiLU(x)
+          outt[r * Ly::SEG + ch] = y;
+          if (r < n) acc += __bfloat162float(y);  // the centroid averages the stored bf16 keys
+        }
+      }
     }
     __syncthreads();
     for (int i = tid; i < n * CPR; i += kThreads) {
