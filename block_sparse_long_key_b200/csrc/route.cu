@@ -24,13 +24,15 @@
 // Thread t owns query row t, which is TMEM lane t: tcgen05.ld hands it that
 // row's NC scores in registers.  Scores above the thread's running threshold
 // (the worst of its current k-1 best) go to a small per-thread candidate
-// buffer in shared memory; the whole warp flushes the buffers together.  The
-// k-1 kept entries form a binary min-heap of 64-bit keys (order-preserving
-// score bits << 32 | ~block index, so a larger key is a better block: higher
-// score, then lower index) in shared memory ([slot][thread], bank-conflict
-// free); admitting a candidate replaces the root and sifts it down a fixed
-// log2(k) levels whatever the data, two levels per step (a sorted list would
-// shift up to k-1 entries, and a warp pays for its slowest lane).  At the
+// buffer in shared memory (predicated stores); the whole warp flushes the
+// buffers together.  The k-1 kept entries form a binary min-heap of 64-bit
+// keys (order-preserving score bits << 32 | ~block index, so a larger key is
+// a better block: higher score, then lower index) in shared memory
+// ([slot][thread], bank-conflict free); admitting a candidate replaces the
+// root and sifts it down a fixed log2(k) levels whatever the data, one level
+// (two loads) per step (a sorted list would shift up to k-1 entries, and a
+// warp pays for its slowest lane).  With four CTAs per SM the candidate
+// stores and admissions are bound by shared-memory bandwidth.  At the
 // end each thread sorts its row's kept block indices in registers and writes
 // the row.
 //
@@ -273,36 +275,12 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
     int pos = 0;
     bool done = !go;
     uint64_t root = key;  // the new minimum: the key itself or the smaller child of the root
-    // Two levels per step: the children and all four grandchildren are
-    // loaded together (none depends on the first decision), which halves the
-    // chain of dependent shared-memory loads.
-    int lvl = 0;
+    // One level per step, two loads each: with 16 selecting warps per SM the
+    // admissions are bound by shared-memory bandwidth, not by the chain of
+    // dependent loads (loading the four grandchildren with the children, two
+    // levels per step, costs 50 % more loads and measured no faster).
 #pragma unroll
-    for (; lvl + 1 < kHeapDepth; lvl += 2) {
-      const int c1 = 2 * pos + 1, g1 = 2 * c1 + 1;
-      const uint64_t a0 = heap[c1 * kSel + tid], a1 = heap[(c1 + 1) * kSel + tid];
-      const uint64_t b0 = heap[g1 * kSel + tid], b1 = heap[(g1 + 1) * kSel + tid];
-      const uint64_t b2 = heap[(g1 + 2) * kSel + tid], b3 = heap[(g1 + 3) * kSel + tid];
-      const bool left = a0 < a1;
-      const uint64_t km = left ? a0 : a1;
-      if (!done && km < key) {
-        heap[pos * kSel + tid] = km;
-        if (lvl == 0) root = km;
-        pos = left ? c1 : c1 + 1;
-      } else {
-        done = true;
-      }
-      const uint64_t d0 = left ? b0 : b2, d1 = left ? b1 : b3;  // children of the chosen child
-      const bool left2 = d0 < d1;
-      const uint64_t km2 = left2 ? d0 : d1;
-      if (!done && km2 < key) {
-        heap[pos * kSel + tid] = km2;
-        pos = 2 * pos + (left2 ? 1 : 2);
-      } else {
-        done = true;
-      }
-    }
-    if (lvl < kHeapDepth) {
+    for (int lvl = 0; lvl < kHeapDepth; ++lvl) {
       const int c1 = 2 * pos + 1;
       const uint64_t k1v = heap[c1 * kSel + tid];
       const uint64_t k2v = heap[(c1 + 1) * kSel + tid];
@@ -312,6 +290,8 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
         heap[pos * kSel + tid] = km;
         if (lvl == 0) root = km;
         pos = left ? c1 : c1 + 1;
+      } else {
+        done = true;
       }
     }
     if (go) {
@@ -363,10 +343,14 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
 #pragma unroll
       for (int e = 0; e < kGroup; ++e) {
         const int col = g * kGroup + e;
-        // Branch-free: slot cnt is free (cnt < kBuf here), so the candidate
-        // is stored either way and only counted when it passes.
-        bk[cnt * kSel + tid] = make_uint2(v[col], (uint32_t)(jbase + col));
-        cnt += __uint_as_float(v[col]) > thr ? 1 : 0;
+        // Predicated store (slot cnt is free: cnt < kBuf here).  Only a few
+        // per cent of the scores pass, and shared-memory bandwidth, shared
+        // with the heap admissions, limits the selection: a lane that does
+        // not store takes no bandwidth.
+        if (__uint_as_float(v[col]) > thr) {
+          bk[cnt * kSel + tid] = make_uint2(v[col], (uint32_t)(jbase + col));
+          ++cnt;
+        }
       }
     }
   };
