@@ -204,7 +204,10 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   // padding slots up to LISTN-1 hold kKeyMax and never surface.
   if (sel_thread)
     for (int sl = 0; sl < LISTN; ++sl) heap[sl * kSel + tid] = sl < k1 ? kKeyEmpty : kKeyMax;
-  uint64_t root_key = kKeyEmpty;  // the heap's root: the worst kept key
+  uint64_t root_key = kKeyEmpty;  // heap slot 0, the root: the worst kept key
+  // Slots 1 and 2 (the root's children) live in registers as well, so an
+  // admission touches shared memory from the third level on.
+  uint64_t h1 = 1 < k1 ? kKeyEmpty : kKeyMax, h2 = 2 < k1 ? kKeyEmpty : kKeyMax;
   float tau = -INFINITY;          // its score
   float lb = -INFINITY;           // the first pass's lower bound (two-pass tiles)
   // Candidates pass when x > thr = max(tau, the float just below lb): x > tau
@@ -272,15 +275,38 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
   // Admits `key` when `go` (branch-free: a thread with nothing to admit
   // walks the same instructions with every store switched off).
   auto admit = [&](uint64_t key, bool go) {
-    int pos = 0;
-    bool done = !go;
-    uint64_t root = key;  // the new minimum: the key itself or the smaller child of the root
-    // One level per step, two loads each: with 16 selecting warps per SM the
-    // admissions are bound by shared-memory bandwidth, not by the chain of
-    // dependent loads (loading the four grandchildren with the children, two
-    // levels per step, costs 50 % more loads and measured no faster).
+    // level 0: the root's children, in registers
+    const bool left0 = h1 < h2;
+    const uint64_t km0 = left0 ? h1 : h2;
+    const bool up0 = go && km0 < key;
+    const uint64_t root = up0 ? km0 : key;  // the new minimum
+    int pos = up0 ? (left0 ? 1 : 2) : 0;
+    bool done = !up0;
+    // level 1: the children of register slot pos (slots 3 .. 6); what moves
+    // up, or the key itself, goes into that register
+    uint64_t r1 = key;
+    {
+      const int c1 = 2 * pos + 1;  // (pos 0: slots 1 and 2 of shared memory, stale and unused)
+      const uint64_t k1v = heap[c1 * kSel + tid];
+      const uint64_t k2v = heap[(c1 + 1) * kSel + tid];
+      const bool left = k1v < k2v;
+      const uint64_t km = left ? k1v : k2v;
+      if (!done && km < key) {
+        r1 = km;
+        pos = left ? c1 : c1 + 1;
+      } else {
+        done = true;
+      }
+    }
+    h1 = up0 && left0 ? r1 : h1;
+    h2 = up0 && !left0 ? r1 : h2;
+    // Deeper levels in shared memory, one level per step, two loads each:
+    // with 16 selecting warps per SM the admissions are bound by
+    // shared-memory bandwidth, not by the chain of dependent loads (loading
+    // the four grandchildren with the children, two levels per step, costs
+    // 50 % more loads and measured no faster).
 #pragma unroll
-    for (int lvl = 0; lvl < kHeapDepth; ++lvl) {
+    for (int lvl = 2; lvl < kHeapDepth; ++lvl) {
       const int c1 = 2 * pos + 1;
       const uint64_t k1v = heap[c1 * kSel + tid];
       const uint64_t k2v = heap[(c1 + 1) * kSel + tid];
@@ -288,14 +314,13 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
       const uint64_t km = left ? k1v : k2v;
       if (!done && km < key) {
         heap[pos * kSel + tid] = km;
-        if (lvl == 0) root = km;
         pos = left ? c1 : c1 + 1;
       } else {
         done = true;
       }
     }
     if (go) {
-      heap[pos * kSel + tid] = key;
+      if (pos >= 3) heap[pos * kSel + tid] = key;  // slots 0 .. 2 took it above
       root_key = root;
       tau = from_order_bits((uint32_t)(root >> 32));
       thr = fmaxf(tau, nextafterf(lb, -INFINITY));
@@ -513,7 +538,8 @@ route_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const __gri
     int kept_n = 0;
 #pragma unroll
     for (int sl = 0; sl < LISTN; ++sl) {
-      const uint64_t key = sl < k1 ? heap[sl * kSel + tid] : kKeyEmpty;
+      const uint64_t key =
+          sl >= k1 ? kKeyEmpty : (sl == 0 ? root_key : (sl == 1 ? h1 : (sl == 2 ? h2 : heap[sl * kSel + tid])));
       const bool real = key != kKeyEmpty;
       kept_n += real;
       ix[sl] = real ? 0xffffffffu - (uint32_t)key : 0x7fffffffu;  // block index; empty slots sort last
