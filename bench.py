@@ -51,11 +51,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel source file it was taken with: a changed source voids the figure.
 # Headline workload, one timed-step launch each (profiles/dram_traffic_n64k_h16_d64_b32_k32_kconv4.md).
 NCU_TRAFFIC = {
-    "fwd_route": {"bytes": 278.22e6 + 366.72e6, "sha": "6cb84cd7d1226227"},
-    "fwd_attn": {"bytes": 1.1706e9 + 719.20e6, "sha": "5b561e1c286c88a7"},
-    "bwd_attn": {"bytes": 1.9063e9 + 1.0038e9, "sha": "3ffdaa36749d5531"},
-    "conv_bwd": {"bytes": 268.46e6 + 127.35e6, "sha": "2e8a64640582a328"},
-    "fwd_centroid": {"bytes": 134.26e6 + 101.85e6, "sha": "103ae9898d36c11f"},
+    "fwd_route": {"bytes": 278.49e6 + 366.52e6, "sha": "98c2c86de5d6b6fb"},
+    "fwd_attn": {"bytes": 1.1745e9 + 721.19e6, "sha": "7a566854044986cd"},
+    "bwd_attn": {"bytes": 1.9201e9 + 1.0060e9, "sha": "3ffdaa36749d5531"},
+    "conv_bwd": {"bytes": 268.57e6 + 127.72e6, "sha": "359b7f65ddabf225"},
+    "fwd_centroid": {"bytes": 134.25e6 + 102.05e6, "sha": "792b201ba3dbf790"},
+    "fwd_index": {"bytes": (134.23e6 + 2.72e6) + 8.40e6 + (172.91e6 + 107.21e6), "sha": "094bee12087fb6be"},
 }
 
 
