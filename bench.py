@@ -366,6 +366,20 @@ def run_ours(args):
     pos = torch.cat([torch.arange(b - a) for a, b in zip(x["cu_seqlens"][:-1].tolist(),
                                                          x["cu_seqlens"][1:].tolist())]).double()
     scored = float((pos // B).sum().item()) * hq
+    # Exact useful work (the nominal count above assumes k full blocks per
+    # row): a past block contributes B keys, the own block the (p mod B) + 1
+    # keys up to the query, and early queries hold fewer than k picks.
+    own_keys = float(((pos % B) + 1).sum().item()) * hq
+    visible_keys = (pairs - T * hq) * B + own_keys
+    useful_fwd = 4.0 * d * visible_keys
+    useful_bwd = 2.5 * useful_fwd
+    # Planted needles (query, head, block) that the router picked.
+    needle_recall = None
+    if x.get("needles"):
+        nd = torch.tensor([[hq_, i_, j_] for _, hq_, i_, j_ in x["needles"]], dtype=torch.long, device=dev)
+        rows_sel = sel[nd[:, 1], nd[:, 0]]
+        picked = int((rows_sel == nd[:, 2:3].to(torch.int32)).any(dim=1).sum().item())
+        needle_recall = {"planted": int(nd.shape[0]), "picked": picked}
 
     stream = torch.cuda.current_stream()
     stage_sets = [moba.StageEvents() for _ in range(args.steps)]
@@ -541,7 +555,14 @@ def run_ours(args):
             "pct_of_bf16_peak": round(100.0 * value / world / peak_t, 3),
             "peak_bf16_tflops": peak_t, "peak_source": peak_src,
             "stage_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
-            "pairs": pairs, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "memory": memory,
+            "pairs": pairs,
+            # rank 0's useful work (its shard, or its replica) times the ranks
+            "useful": {"visible_keys": int(visible_keys), "of_nominal": round(visible_keys / (T * hq * topk * B), 4),
+                       "fwd_tflops": round(useful_fwd / (fwd_ms * 1e-3) / 1e12, 3),
+                       "bwd_tflops": round(useful_bwd / (bwd_ms * 1e-3) / 1e12, 3),
+                       "step_tflops": round(aggregate_value((useful_fwd + useful_bwd) * world, ms_max), 3)},
+            "needle_recall": needle_recall,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "memory": memory,
             "dense_context": dense,
             "gpu_launches": (LAUNCHES_PER_STEP + (LAUNCHES_CONV_BWD if w.conv_width else 0)) * args.steps, "clocks": clocks.summary(), "device_status": status,
         }
