@@ -28,6 +28,12 @@ SMALL = [
     ((2500, 77), 4, 1, 64, 16, 6, 0),               # GQA 4:1, B=16: buckets of many 128-row tiles
 ]
 
+# Key-conv widths beyond the SMALL cases (the register windows of both conv
+# kernels are unrolled per width): ragged sequences, blocks shorter than and
+# equal to twice the halo.
+CONV_WIDTHS = [((300, 5, 700), 2, 2, 64, 32, 4, W) for W in (1, 2, 6, 7, 8)] + \
+    [((260, 33), 2, 1, 128, 16, 3, 8)]
+
 
 def _ids(c):
     return "L%s_h%dx%d_d%d_B%d_k%d_w%d" % ("-".join(map(str, c[0])), c[1], c[2], c[3], c[4], c[5], c[6])
@@ -77,7 +83,7 @@ def test_forward_matches_oracle(dev, case):
     pu.check_o_lse(o_g, lse_g, o_ref, lse_ref, _ids(case))
 
 
-@pytest.mark.parametrize("case", [c for c in SMALL if c[6] > 0] + [SMALL[1]], ids=_ids)
+@pytest.mark.parametrize("case", [c for c in SMALL if c[6] > 0] + [SMALL[1]] + CONV_WIDTHS, ids=_ids)
 def test_conv_and_centroids_match_oracle(dev, case):
     w, x = _inputs(case)
     g = _gpu(x, dev)
@@ -364,7 +370,7 @@ def test_backward_reusing_forward_index_matches_oracle(dev, case):
     pu.check_grad(pu.to64(dv), dv_r, sv, "dv reuse")
 
 
-@pytest.mark.parametrize("case", [SMALL[3], SMALL[7], ((300, 5, 700), 2, 2, 128, 16, 4, 5)], ids=_ids)
+@pytest.mark.parametrize("case", [SMALL[3], SMALL[7], ((300, 5, 700), 2, 2, 128, 16, 4, 5)] + CONV_WIDTHS, ids=_ids)
 def test_key_conv_backward_matches_oracle(dev, case):
     w, x = _inputs(case)
     g = _gpu(x, dev)
