@@ -136,10 +136,11 @@ fill_kernel(const int32_t* __restrict__ sel_idx, long long npicks, int topk, int
 // ---- shared-memory privatised path
 //
 // A CTA owns the picks of one (chunk of kChunkTokens tokens, KV head).  The
-// count and the staged fill take one pick per thread and step (coalesced
-// loads, several independent picks in flight per thread); the unstaged fill
-// takes one query row per thread and walks its topk picks.  The per-pick
-// work is a load, a range check and one shared-memory atomic.
+// count and the staged fill take a run of kRun consecutive slots of one
+// query row per thread (coalesced loads, several picks in flight per
+// thread); the unstaged fill takes one query row per thread and walks its
+// topk picks.  The per-pick work is a load, a range check and one
+// shared-memory atomic.
 
 // For query row `r` of the chunk (ta: first token): its row id, its
 // sequence's first global block and its own block; false past the chunk or
