@@ -17,8 +17,9 @@
 // to the pending outputs of t = u - l and emits dK_t into a shared output
 // tile once u = t + W - 1; the tile leaves with 16-byte coalesced stores.
 // Its block's dW partial goes to a per-block buffer that a second kernel sums
-// over blocks in a fixed order (deterministic).  HBM-bound: K and dK' read
-// once (plus the halo rows), dK written once.
+// over blocks in a fixed order (deterministic).  Traffic: K and dK' read
+// once (plus the halo rows), dK written once; the walk itself (about 30
+// instructions per element with the register rings below) sets the time.
 #include "common.cuh"
 #include "launch.h"
 
