@@ -54,9 +54,9 @@ NCU_TRAFFIC = {
     "fwd_route": {"bytes": 278.49e6 + 366.52e6, "sha": "98c2c86de5d6b6fb"},
     "fwd_attn": {"bytes": 1.1745e9 + 721.19e6, "sha": "7a566854044986cd"},
     "bwd_attn": {"bytes": 1.9201e9 + 1.0060e9, "sha": "3ffdaa36749d5531"},
-    "conv_bwd": {"bytes": 268.57e6 + 127.72e6, "sha": "359b7f65ddabf225"},
+    "conv_bwd": {"bytes": 268.57e6 + 127.72e6, "sha": "cab0cb4e397e800e"},
     "fwd_centroid": {"bytes": 134.25e6 + 102.05e6, "sha": "792b201ba3dbf790"},
-    "fwd_index": {"bytes": (134.23e6 + 2.72e6) + 8.40e6 + (172.91e6 + 107.21e6), "sha": "094bee12087fb6be"},
+    "fwd_index": {"bytes": (134.23e6 + 2.72e6) + 8.40e6 + (172.91e6 + 107.21e6), "sha": "4a2d500ca215863b"},
 }
 
 
