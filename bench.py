@@ -160,6 +160,16 @@ def rank_seed(w: synth.Workload, rank: int) -> int:
     return w.seed + 7919 * rank
 
 
+def visible_keys(pos: "torch.Tensor", block_size: int, h_q: int, pairs: int) -> float:
+    """Keys the attention actually reads, summed over every (query, head):
+    `pairs` valid picks (own block included, one per query and head), each
+    past block contributing B keys and the own block the (p mod B) + 1 keys
+    up to the query at in-sequence position p.  The nominal count assumes k
+    full blocks per query and head."""
+    own = float(((pos % block_size) + 1).sum().item()) * h_q
+    return (pairs - pos.numel() * h_q) * block_size + own
+
+
 def head_shard(h_kv: int, world: int, rank: int):
     """KV heads [kv0, kv1) of rank `rank` when one problem's KV-head groups
     are split over `world` ranks: contiguous ranges, the first h_kv % world
@@ -369,9 +379,8 @@ def run_ours(args):
     # Exact useful work (the nominal count above assumes k full blocks per
     # row): a past block contributes B keys, the own block the (p mod B) + 1
     # keys up to the query, and early queries hold fewer than k picks.
-    own_keys = float(((pos % B) + 1).sum().item()) * hq
-    visible_keys = (pairs - T * hq) * B + own_keys
-    useful_fwd = 4.0 * d * visible_keys
+    n_visible = visible_keys(pos, B, hq, pairs)
+    useful_fwd = 4.0 * d * n_visible
     useful_bwd = 2.5 * useful_fwd
     # Planted needles (query, head, block) that the router picked.
     needle_recall = None
@@ -557,7 +566,7 @@ def run_ours(args):
             "stage_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
             "pairs": pairs,
             # rank 0's useful work (its shard, or its replica) times the ranks
-            "useful": {"visible_keys": int(visible_keys), "of_nominal": round(visible_keys / (T * hq * topk * B), 4),
+            "useful": {"visible_keys": int(n_visible), "of_nominal": round(n_visible / (T * hq * topk * B), 4),
                        "fwd_tflops": round(useful_fwd / (fwd_ms * 1e-3) / 1e12, 3),
                        "bwd_tflops": round(useful_bwd / (bwd_ms * 1e-3) / 1e12, 3),
                        "step_tflops": round(aggregate_value((useful_fwd + useful_bwd) * world, ms_max), 3)},
